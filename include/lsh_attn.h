@@ -1,0 +1,151 @@
+/*
+ * lsh_attn.h -- C ABI of the B200 (sm_100a) Reformer shared-QK LSH-attention
+ * forward pass.
+ *
+ * The method (sources are web pages on Reformer, cited by title and section):
+ *   - hash: for b buckets a random R of size [dimension, b/2] maps x to
+ *     argmax([xR ; -xR])                  ("Reformer summary", §局部敏感哈希)
+ *   - several independent hash rounds     ("Reformer summary", §多輪LSH哈希)
+ *   - sort the tokens by bucket, then by position; cut the sorted order into
+ *     chunks of m and attend inside them  ("Reformer summary", §局部敏感哈希注意力)
+ *   - keys are the shared vectors scaled to unit length, logits are scaled by
+ *     1/sqrt(d) ("Reformer: LSH attention and reversible layers", §二.1)
+ *   - a token attends to itself only when nothing else is available
+ *                                         ("Reformer summary", §共享QK中的自掩碼)
+ * Readings taken where the pages are silent: a query in chunk c sees the keys
+ * of chunks c-1 and c (chunk 0 sees only itself); the self logit is -1e5;
+ * causal masking removes keys at later positions; rounds are merged by
+ * weighting each round's output with exp(lse_r - logsumexp_r lse_r); argmax
+ * ties go to the first index of [xR ; -xR].
+ *
+ * Conventions for every entry point
+ *   - All array pointers are DEVICE pointers owned by the caller. The library
+ *     never allocates device memory; scratch space is the caller's workspace of
+ *     at least lsh_attn_workspace_size() bytes, 256-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronise the host, except
+ *     lsh_attn_get_device_status / lsh_attn_get_diag, which synchronise
+ *     `stream`.
+ *   - Argument errors are detected on the host before anything is launched;
+ *     nothing is written then. Errors found by the kernels (a caller bucket id
+ *     outside [0, n_buckets), a bounded wait that gave up) are recorded in the
+ *     workspace status word and read with lsh_attn_get_device_status.
+ *   - Results are deterministic: identical inputs give bit-identical outputs.
+ *   - One workspace must not be shared by calls that may run concurrently.
+ *
+ * Layouts (row-major, innermost last; B batch, H heads, n length, d head
+ * dim, nb buckets, Rn rounds):
+ *   x, v, out    [B][H][n][d]          in desc.dtype
+ *   R            [Rn][d][nb/2]         in desc.dtype
+ *   buckets      [B][H][Rn][n]         int32, position order
+ *   perm         [B][H][Rn][n]         int32: perm[s] = position at sorted slot s
+ *   xs, vs       [B][H][Rn][n][d]      desc.dtype, rows in sorted order
+ *   lse          [B][H][Rn][n]         fp32, position order, natural log
+ *
+ * Supported (else LSH_ERR_UNSUPPORTED): dtype LSH_F32 or LSH_BF16; d in
+ * {64, 128}; n_buckets even with 2 <= n_buckets <= 4096; chunk m >= 1 with
+ * min(m, n) <= 128 and n % min(m, n) == 0 (m >= n is a single chunk);
+ * 1 <= rounds <= 16; n * n_buckets < 2^31.
+ */
+#ifndef LSH_ATTN_H
+#define LSH_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LSH_OK = 0,
+    LSH_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad enum */
+    LSH_ERR_UNSUPPORTED = 2, /* a valid problem outside the supported set */
+    LSH_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
+    LSH_ERR_CUDA = 4,        /* a CUDA runtime call failed */
+    LSH_ERR_TIMEOUT = 5,     /* a kernel's bounded wait gave up */
+    LSH_ERR_DEVICE = 6       /* a kernel rejected its input (bucket id range) */
+} lsh_status;
+
+typedef enum { LSH_F32 = 0, LSH_BF16 = 1 } lsh_dtype;
+
+/* Problem description shared by every call. */
+typedef struct {
+    int32_t batch;     /* B >= 1 */
+    int32_t heads;     /* H >= 1 */
+    int32_t n;         /* sequence length >= 1 */
+    int32_t d;         /* head dimension */
+    int32_t n_buckets; /* nb: even, buckets per round */
+    int32_t chunk;     /* m: chunk length in the sorted order */
+    int32_t rounds;    /* independent hash rounds */
+    int32_t causal;    /* 0 or 1 */
+    int32_t dtype;     /* lsh_dtype of x, v, R, out, xs, vs */
+} lsh_attn_desc;
+
+/* Counters written by the kernels into the workspace header; reset at the
+ * start of every hash / sort / forward call. */
+typedef struct {
+    uint32_t status;         /* lsh_status recorded by a kernel, 0 if none */
+    uint32_t hash_refined;   /* (token, round) hashes re-decided in fp64 */
+    uint32_t bad_bucket_ids; /* caller bucket ids outside [0, nb), clamped */
+    uint32_t reserved;
+} lsh_attn_diag;
+
+/* Workspace bytes that lsh_attn_hash / lsh_attn_sort / lsh_attn_forward need
+ * for `desc`. Writes *bytes; errors as for the calls themselves. */
+lsh_status lsh_attn_workspace_size(const lsh_attn_desc *desc, size_t *bytes);
+
+/* Hash every token in every round ("Reformer summary", §局部敏感哈希 and
+ * §多輪LSH哈希): buckets[b][h][r][i] = argmax([x_i R_r ; -x_i R_r]), first
+ * index on ties, bit-exact to the fp64 definition (bf16 runs on tensor cores
+ * and re-decides near ties in fp64; fp32 runs in fp64).
+ * x [B][H][n][d], R [Rn][d][nb/2] in desc.dtype; buckets out, int32. */
+lsh_status lsh_attn_hash(const lsh_attn_desc *desc, const void *x, const void *R,
+                         int32_t *buckets, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/* Stable sort of every (batch, head, round) by bucket, then position
+ * ("Reformer summary", §局部敏感哈希注意力): perm[s] = the position at sorted
+ * slot s. If x, v, xs and vs are all non-NULL the rows of x and v are also
+ * gathered into sorted order: xs[..][s] = x[..][perm[s]]; pass all four NULL
+ * to skip the gather. buckets [B][H][Rn][n] int32 in [0, nb) (ids outside are
+ * clamped and counted in the diag). */
+lsh_status lsh_attn_sort(const lsh_attn_desc *desc, const int32_t *buckets, const void *x,
+                         const void *v, int32_t *perm, void *xs, void *vs, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/* Whole forward pass: hash (skipped when `buckets` is non-NULL: the caller's
+ * ids are used as given), sort and gather, chunked attention with unit keys,
+ * 1/sqrt(d) scale, optional causal mask and the -1e5 self logit, un-sort, and
+ * the logsumexp round merge. out [B][H][n][d] in desc.dtype; lse [B][H][Rn][n]
+ * fp32 holds every round's log-normaliser in position order. */
+lsh_status lsh_attn_forward(const lsh_attn_desc *desc, const void *x, const void *v,
+                            const void *R, const int32_t *buckets, void *out, float *lse,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* lsh_attn_forward that also records the caller's CUDA events on `stream`
+ * at the stage boundaries, for timing each stage on the device:
+ *   events[0] before the hash      events[1] after the hash (right after
+ *   events[0] when buckets are given)   events[2] after the sort and gather
+ *   events[3] after the chunked attention   events[4] after the round merge.
+ * `events` points to 5 cudaEvent_t handles created by the caller. */
+lsh_status lsh_attn_forward_profiled(const lsh_attn_desc *desc, const void *x, const void *v,
+                                     const void *R, const int32_t *buckets, void *out, float *lse,
+                                     void *workspace, size_t workspace_bytes, void *stream,
+                                     void *const *events);
+
+/* Synchronise `stream` and return the status the kernels recorded in
+ * `workspace` since the last call that used it (LSH_OK if none). */
+lsh_status lsh_attn_get_device_status(const void *workspace, void *stream);
+
+/* Synchronise `stream` and copy the workspace counters into *diag. */
+lsh_status lsh_attn_get_diag(const void *workspace, void *stream, lsh_attn_diag *diag);
+
+/* Static, human-readable name of a status code. */
+const char *lsh_attn_status_string(lsh_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSH_ATTN_H */

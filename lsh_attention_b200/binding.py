@@ -1,0 +1,229 @@
+"""Thin Python binding of the C ABI in include/lsh_attn.h.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library liblshattn.so. PyTorch supplies device memory (inputs, outputs and
+the workspace) and the current CUDA stream. There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblshattn.so")
+
+LSH_F32, LSH_BF16 = 0, 1
+_DTYPES = {torch.float32: LSH_F32, torch.bfloat16: LSH_BF16}
+
+#: every symbol the header declares
+EXPORTS = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_forward",
+           "lsh_attn_forward_profiled", "lsh_attn_get_device_status", "lsh_attn_get_diag",
+           "lsh_attn_status_string")
+
+
+class LshAttnDesc(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_int32) for k in
+                ("batch", "heads", "n", "d", "n_buckets", "chunk", "rounds", "causal", "dtype")]
+
+
+class LshAttnDiag(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_uint32) for k in
+                ("status", "hash_refined", "bad_bucket_ids", "reserved")]
+
+
+class LshAttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load() -> ctypes.CDLL:
+    """Load liblshattn.so; raise if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                                  "`python -m lsh_attention_b200.build`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            vp, sz = ctypes.c_void_p, ctypes.c_size_t
+            dp = ctypes.POINTER(LshAttnDesc)
+            lib.lsh_attn_workspace_size.argtypes = [dp, ctypes.POINTER(sz)]
+            lib.lsh_attn_hash.argtypes = [dp, vp, vp, vp, vp, sz, vp]
+            lib.lsh_attn_sort.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            lib.lsh_attn_forward.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            lib.lsh_attn_forward_profiled.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                                      ctypes.POINTER(ctypes.c_void_p)]
+            lib.lsh_attn_get_device_status.argtypes = [vp, vp]
+            lib.lsh_attn_get_diag.argtypes = [vp, vp, ctypes.POINTER(LshAttnDiag)]
+            lib.lsh_attn_status_string.argtypes = [ctypes.c_int]
+            lib.lsh_attn_status_string.restype = ctypes.c_char_p
+            for f in EXPORTS[:-1]:
+                getattr(lib, f).restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        msg = load().lsh_attn_status_string(status).decode()
+        raise LshAttnError(status, msg)
+
+
+def make_desc(batch, heads, n, d, n_buckets, chunk, rounds, causal, dtype) -> LshAttnDesc:
+    if isinstance(dtype, torch.dtype):
+        if dtype not in _DTYPES:
+            raise TypeError(f"unsupported dtype {dtype}")
+        dtype = _DTYPES[dtype]
+    return LshAttnDesc(batch, heads, n, d, n_buckets, chunk, rounds, int(bool(causal)), dtype)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _require(t: torch.Tensor, name: str, dtype, shape) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def lsh_attn_workspace_size(desc: LshAttnDesc) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load().lsh_attn_workspace_size(ctypes.byref(desc), ctypes.byref(out)))
+    return out.value
+
+
+_ws_cache: dict = {}
+
+
+def workspace(desc: LshAttnDesc, device, stream=None) -> torch.Tensor:
+    """A cached workspace of at least the size `desc` needs, one per
+    (device, stream): calls that may run concurrently must not share one."""
+    need = lsh_attn_workspace_size(desc)
+    dev = torch.device(device)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    key = (dev.index, s.cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        _ws_cache.pop(key, None)
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        _ws_cache[key] = ws
+    return ws
+
+
+def lsh_attn_hash(x, R, n_buckets: int, buckets=None, ws=None, stream=None):
+    """Bucket ids [B, H, rounds, n] int32 of x [B, H, n, d] under R [rounds, d, nb/2]."""
+    B, H, n, d = x.shape
+    rounds = R.shape[0]
+    _require(x, "x", None, None)
+    _require(R, "R", x.dtype, (rounds, d, n_buckets // 2))
+    desc = make_desc(B, H, n, d, n_buckets, 1, rounds, False, x.dtype)
+    if buckets is None:
+        buckets = torch.empty((B, H, rounds, n), dtype=torch.int32, device=x.device)
+    _require(buckets, "buckets", torch.int32, (B, H, rounds, n))
+    if ws is None:
+        ws = workspace(desc, x.device, stream)
+    _check(load().lsh_attn_hash(ctypes.byref(desc), _ptr(x), _ptr(R), _ptr(buckets), _ptr(ws),
+                                ws.numel(), _stream(stream)))
+    return buckets
+
+
+def lsh_attn_sort(buckets, n_buckets: int, x=None, v=None, perm=None, xs=None, vs=None, ws=None,
+                  stream=None, d: int = 64, dtype=torch.bfloat16):
+    """Stable sort by (bucket, position) of every (batch, head, round).
+    Returns perm [B, H, rounds, n] int32, and (xs, vs) sorted row copies when
+    x and v are given."""
+    B, H, rounds, n = buckets.shape
+    _require(buckets, "buckets", torch.int32, None)
+    if x is not None:
+        _require(x, "x", None, (B, H, n, x.shape[-1]))
+        _require(v, "v", x.dtype, tuple(x.shape))
+        d, dtype = x.shape[-1], x.dtype
+    desc = make_desc(B, H, n, d, n_buckets, 1, rounds, False, dtype)
+    if perm is None:
+        perm = torch.empty((B, H, rounds, n), dtype=torch.int32, device=buckets.device)
+    _require(perm, "perm", torch.int32, (B, H, rounds, n))
+    if x is not None:
+        if xs is None:
+            xs = torch.empty((B, H, rounds, n, d), dtype=dtype, device=x.device)
+        if vs is None:
+            vs = torch.empty((B, H, rounds, n, d), dtype=dtype, device=x.device)
+        _require(xs, "xs", dtype, (B, H, rounds, n, d))
+        _require(vs, "vs", dtype, (B, H, rounds, n, d))
+    if ws is None:
+        ws = workspace(desc, buckets.device, stream)
+    _check(load().lsh_attn_sort(ctypes.byref(desc), _ptr(buckets), _ptr(x), _ptr(v), _ptr(perm),
+                                _ptr(xs), _ptr(vs), _ptr(ws), ws.numel(), _stream(stream)))
+    return (perm, xs, vs) if x is not None else perm
+
+
+def lsh_attn_forward(x, v, R=None, *, n_buckets: int, chunk: int, causal: bool, rounds=None,
+                     buckets=None, out=None, lse=None, ws=None, stream=None, events=None):
+    """LSH-attention forward. x, v [B, H, n, d]; R [rounds, d, nb/2] (or
+    caller buckets [B, H, rounds, n]). Returns (out [B, H, n, d], lse
+    [B, H, rounds, n] fp32). `events`: five recorded torch.cuda.Event objects
+    to mark the stage boundaries (lsh_attn_forward_profiled)."""
+    B, H, n, d = x.shape
+    _require(x, "x", None, None)
+    _require(v, "v", x.dtype, tuple(x.shape))
+    if buckets is not None:
+        rounds = buckets.shape[2]
+        _require(buckets, "buckets", torch.int32, (B, H, rounds, n))
+    else:
+        if R is None:
+            raise ValueError("either R or buckets is required")
+        rounds = R.shape[0]
+        _require(R, "R", x.dtype, (rounds, d, n_buckets // 2))
+    desc = make_desc(B, H, n, d, n_buckets, chunk, rounds, causal, x.dtype)
+    if out is None:
+        out = torch.empty_like(x)
+    if lse is None:
+        lse = torch.empty((B, H, rounds, n), dtype=torch.float32, device=x.device)
+    _require(out, "out", x.dtype, tuple(x.shape))
+    _require(lse, "lse", torch.float32, (B, H, rounds, n))
+    if ws is None:
+        ws = workspace(desc, x.device, stream)
+    args = (ctypes.byref(desc), _ptr(x), _ptr(v), _ptr(R), _ptr(buckets), _ptr(out), _ptr(lse),
+            _ptr(ws), ws.numel(), _stream(stream))
+    if events is None:
+        _check(load().lsh_attn_forward(*args))
+    else:
+        if len(events) != 5 or any(e.cuda_event == 0 for e in events):
+            raise ValueError("events: five torch.cuda.Event objects, each recorded once")
+        ev = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+        _check(load().lsh_attn_forward_profiled(*args, ev))
+    return out, lse
+
+
+def lsh_attn_get_diag(ws, stream=None) -> dict:
+    d = LshAttnDiag()
+    _check(load().lsh_attn_get_diag(_ptr(ws), _stream(stream), ctypes.byref(d)))
+    return {"status": d.status, "hash_refined": d.hash_refined,
+            "bad_bucket_ids": d.bad_bucket_ids}
+
+
+def lsh_attn_get_device_status(ws, stream=None) -> int:
+    return load().lsh_attn_get_device_status(_ptr(ws), _stream(stream))

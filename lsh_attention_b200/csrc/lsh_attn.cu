@@ -1,0 +1,334 @@
+// Host side of the C ABI declared in include/lsh_attn.h: argument checks,
+// workspace carving, and kernel launches on the caller's stream.
+#include "lsh_attn.h"
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "attn_simt.cuh"
+#include "common.cuh"
+#include "hash_exact.cuh"
+#include "merge.cuh"
+#include "sort.cuh"
+
+namespace {
+
+using namespace lsh;
+
+struct Layout {
+  size_t header, buckets, perm, inv, invnorm, lse_s, hist, xs, vs, out_s, total;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Dims {
+  int B, H, n, d, nb, m, rounds, causal, dtype;
+  int64_t BH, S;  // (batch, head) pairs; segments = BH * rounds
+  int esize;
+  int tiles;
+};
+
+// `attention`: the call runs the chunked attention, so the chunk length must
+// be in the supported set; hash and sort ignore it beyond chunk >= 1.
+lsh_status check_desc(const lsh_attn_desc* desc, Dims* D, bool attention) {
+  if (!desc) return LSH_ERR_INVALID_ARG;
+  const lsh_attn_desc& q = *desc;
+  if (q.batch < 1 || q.heads < 1 || q.n < 1 || q.d < 1 || q.n_buckets < 1 || q.chunk < 1 ||
+      q.rounds < 1 || (q.causal != 0 && q.causal != 1) || (q.dtype != LSH_F32 && q.dtype != LSH_BF16))
+    return LSH_ERR_INVALID_ARG;
+  if (q.d != 64 && q.d != 128) return LSH_ERR_UNSUPPORTED;
+  if (q.n_buckets % 2 != 0 || q.n_buckets < 2 || q.n_buckets > 4096) return LSH_ERR_UNSUPPORTED;
+  if (q.rounds > 16) return LSH_ERR_UNSUPPORTED;
+  const int m = q.chunk < q.n ? q.chunk : q.n;
+  if (attention && (m > 128 || q.n % m != 0)) return LSH_ERR_UNSUPPORTED;
+  if ((int64_t)q.n * q.n_buckets >= (int64_t(1) << 31)) return LSH_ERR_UNSUPPORTED;
+  D->B = q.batch;
+  D->H = q.heads;
+  D->n = q.n;
+  D->d = q.d;
+  D->nb = q.n_buckets;
+  D->m = m;
+  D->rounds = q.rounds;
+  D->causal = q.causal;
+  D->dtype = q.dtype;
+  D->BH = (int64_t)q.batch * q.heads;
+  D->S = D->BH * q.rounds;
+  D->esize = q.dtype == LSH_BF16 ? 2 : 4;
+  const int tile = sort_tile(q.n_buckets);
+  D->tiles = (q.n + tile - 1) / tile;
+  if (D->S * (int64_t)q.n * q.d >= (int64_t(1) << 40)) return LSH_ERR_UNSUPPORTED;
+  if (D->S > 65535) return LSH_ERR_UNSUPPORTED;  // segments index grid.y
+  return LSH_OK;
+}
+
+Layout layout_of(const Dims& D) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const size_t sn = (size_t)D.S * D.n;
+  L.header = take(sizeof(WsHeader));
+  L.buckets = take(sn * 4);
+  L.perm = take(sn * 4);
+  L.inv = take(sn * 4);
+  L.invnorm = take(sn * 4);
+  L.lse_s = take(sn * 4);
+  L.hist = take((size_t)D.S * D.nb * D.tiles * 4);
+  L.xs = take(sn * D.d * D.esize);
+  L.vs = take(sn * D.d * D.esize);
+  L.out_s = take(sn * D.d * 4);
+  L.total = off;
+  return L;
+}
+
+lsh_status check_ws(const Dims& D, const void* ws, size_t ws_bytes, Layout* L) {
+  *L = layout_of(D);
+  if (!ws || ((uintptr_t)ws & 255) != 0 || ws_bytes < L->total) return LSH_ERR_WORKSPACE;
+  return LSH_OK;
+}
+
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+inline lsh_status last_cuda() {
+  return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<unsigned char*>(ws) + off);
+}
+
+lsh_status reset_header(void* ws, cudaStream_t st) {
+  return cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- launches
+template <typename T>
+lsh_status launch_hash(const Dims& D, const void* x, const void* R, int32_t* buckets,
+                       cudaStream_t st) {
+  const int xstride = D.d + (sizeof(T) == 4 ? 1 : 2);
+  const size_t smem = sizeof(double) * D.d * kHashExactCols +
+                      sizeof(T) * (size_t)kHashExactTokens * xstride;
+  auto kern = k_hash_exact<T>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LSH_ERR_CUDA;
+  dim3 grid((D.n + kHashExactTokens - 1) / kHashExactTokens, (unsigned)D.BH, D.rounds);
+  kern<<<grid, kHashExactTokens, smem, st>>>(static_cast<const T*>(x), static_cast<const T*>(R),
+                                              buckets, D.n, D.d, D.nb, D.rounds);
+  return last_cuda();
+}
+
+template <typename T>
+lsh_status launch_sort(const Dims& D, const int32_t* buckets, const void* x, const void* v,
+                       int32_t* perm, int32_t* inv, void* xs, void* vs, float* invnorm,
+                       int32_t* hist, WsHeader* hdr, cudaStream_t st) {
+  const int tile = sort_tile(D.nb);
+  dim3 grid(D.tiles, (unsigned)D.S);
+  k_sort_hist<<<grid, 256, sizeof(int32_t) * D.nb, st>>>(buckets, D.n, D.nb, tile, D.tiles, hist,
+                                                         hdr);
+  k_sort_scan<<<(unsigned)D.S, 1024, 0, st>>>(hist, D.nb * D.tiles);
+  const int nw = sort_warps(D.nb);
+  const size_t smem = sizeof(int32_t) * (size_t)nw * D.nb;
+  auto kern = k_sort_scatter<T>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LSH_ERR_CUDA;
+  kern<<<grid, nw * 32, smem, st>>>(buckets, hist, static_cast<const T*>(x),
+                                     static_cast<const T*>(v), perm, inv, static_cast<T*>(xs),
+                                     static_cast<T*>(vs), invnorm, D.n, D.d, D.nb, D.rounds,
+                                     D.tiles);
+  return last_cuda();
+}
+
+template <typename T, int DD, int QPW>
+lsh_status launch_attn_simt_q(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
+                              const float* invnorm, float* out_s, float* lse_s, cudaStream_t st) {
+  const size_t smem = attn_simt_smem(DD);
+  auto kern = k_attn_simt<T, DD, QPW>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LSH_ERR_CUDA;
+  dim3 grid(D.n / D.m, (unsigned)D.S);
+  kern<<<grid, kSimtWarps * 32, smem, st>>>(static_cast<const T*>(xs), static_cast<const T*>(vs),
+                                             perm, invnorm, out_s, lse_s, D.n, D.m, D.causal);
+  return last_cuda();
+}
+
+template <typename T, int DD>
+lsh_status launch_attn_simt(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
+                            const float* invnorm, float* out_s, float* lse_s, cudaStream_t st) {
+  if (D.m <= 16) return launch_attn_simt_q<T, DD, 2>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
+  if (D.m <= 32) return launch_attn_simt_q<T, DD, 4>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
+  if (D.m <= 64) return launch_attn_simt_q<T, DD, 8>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
+  return launch_attn_simt_q<T, DD, 16>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
+}
+
+template <typename T, int DD>
+lsh_status launch_merge(const Dims& D, const int32_t* inv, const float* lse_s, const float* out_s,
+                        void* out, float* lse, cudaStream_t st) {
+  const int64_t total = D.BH * D.n;
+  const unsigned blocks = (unsigned)((total + kMergeWarps - 1) / kMergeWarps);
+  k_merge<T, DD><<<blocks, kMergeWarps * 32, 0, st>>>(inv, lse_s, out_s, static_cast<T*>(out),
+                                                        lse, D.n, D.rounds, total);
+  return last_cuda();
+}
+
+// Record events[i] (if any) on the stream.
+inline lsh_status mark(void* const* events, int i, cudaStream_t st) {
+  if (!events) return LSH_OK;
+  return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess ? LSH_OK
+                                                                              : LSH_ERR_CUDA;
+}
+
+template <typename T>
+lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const void* v,
+                         const void* R, const int32_t* buckets, void* out, float* lse, void* ws,
+                         cudaStream_t st, void* const* ev) {
+  WsHeader* hdr = at<WsHeader>(ws, L.header);
+  lsh_status s;
+  if ((s = mark(ev, 0, st)) != LSH_OK) return s;
+  if (!buckets) {
+    int32_t* bk = at<int32_t>(ws, L.buckets);
+    if ((s = launch_hash<T>(D, x, R, bk, st)) != LSH_OK) return s;
+    buckets = bk;
+  }
+  if ((s = mark(ev, 1, st)) != LSH_OK) return s;
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  float* invnorm = at<float>(ws, L.invnorm);
+  void* xs = at<unsigned char>(ws, L.xs);
+  void* vs = at<unsigned char>(ws, L.vs);
+  float* out_s = at<float>(ws, L.out_s);
+  float* lse_s = at<float>(ws, L.lse_s);
+  if ((s = launch_sort<T>(D, buckets, x, v, perm, inv, xs, vs, invnorm, at<int32_t>(ws, L.hist),
+                          hdr, st)) != LSH_OK)
+    return s;
+  if ((s = mark(ev, 2, st)) != LSH_OK) return s;
+  s = D.d == 64 ? launch_attn_simt<T, 64>(D, xs, vs, perm, invnorm, out_s, lse_s, st)
+                : launch_attn_simt<T, 128>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
+  if (s != LSH_OK) return s;
+  if ((s = mark(ev, 3, st)) != LSH_OK) return s;
+  s = D.d == 64 ? launch_merge<T, 64>(D, inv, lse_s, out_s, out, lse, st)
+                : launch_merge<T, 128>(D, inv, lse_s, out_s, out, lse, st);
+  if (s != LSH_OK) return s;
+  return mark(ev, 4, st);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ C ABI
+extern "C" {
+
+const char* lsh_attn_status_string(lsh_status s) {
+  switch (s) {
+    case LSH_OK: return "LSH_OK";
+    case LSH_ERR_INVALID_ARG: return "LSH_ERR_INVALID_ARG: invalid argument";
+    case LSH_ERR_UNSUPPORTED: return "LSH_ERR_UNSUPPORTED: problem outside the supported set";
+    case LSH_ERR_WORKSPACE: return "LSH_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case LSH_ERR_CUDA: return "LSH_ERR_CUDA: a CUDA runtime call failed";
+    case LSH_ERR_TIMEOUT: return "LSH_ERR_TIMEOUT: a bounded wait in a kernel gave up";
+    case LSH_ERR_DEVICE: return "LSH_ERR_DEVICE: a kernel rejected its input";
+  }
+  return "unknown lsh_status";
+}
+
+lsh_status lsh_attn_workspace_size(const lsh_attn_desc* desc, size_t* bytes) {
+  Dims D;
+  lsh_status s = check_desc(desc, &D, true);
+  if (s != LSH_OK) return s;
+  if (!bytes) return LSH_ERR_INVALID_ARG;
+  *bytes = layout_of(D).total;
+  return LSH_OK;
+}
+
+lsh_status lsh_attn_hash(const lsh_attn_desc* desc, const void* x, const void* R,
+                         int32_t* buckets, void* ws, size_t ws_bytes, void* stream) {
+  Dims D;
+  Layout L;
+  lsh_status s = check_desc(desc, &D, false);
+  if (s != LSH_OK) return s;
+  if (!x || !R || !buckets) return LSH_ERR_INVALID_ARG;
+  if ((s = check_ws(D, ws, ws_bytes, &L)) != LSH_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = reset_header(ws, st)) != LSH_OK) return s;
+  return D.dtype == LSH_BF16 ? launch_hash<__nv_bfloat16>(D, x, R, buckets, st)
+                             : launch_hash<float>(D, x, R, buckets, st);
+}
+
+lsh_status lsh_attn_sort(const lsh_attn_desc* desc, const int32_t* buckets, const void* x,
+                         const void* v, int32_t* perm, void* xs, void* vs, void* ws,
+                         size_t ws_bytes, void* stream) {
+  Dims D;
+  Layout L;
+  lsh_status s = check_desc(desc, &D, false);
+  if (s != LSH_OK) return s;
+  if (!buckets || !perm) return LSH_ERR_INVALID_ARG;
+  const bool gather = x || v || xs || vs;
+  if (gather && (!x || !v || !xs || !vs)) return LSH_ERR_INVALID_ARG;
+  if (gather && !(aligned16(x) && aligned16(v) && aligned16(xs) && aligned16(vs)))
+    return LSH_ERR_INVALID_ARG;
+  if ((s = check_ws(D, ws, ws_bytes, &L)) != LSH_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = reset_header(ws, st)) != LSH_OK) return s;
+  WsHeader* hdr = at<WsHeader>(ws, L.header);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  float* invnorm = at<float>(ws, L.invnorm);
+  int32_t* hist = at<int32_t>(ws, L.hist);
+  if (D.dtype == LSH_BF16)
+    return launch_sort<__nv_bfloat16>(D, buckets, x, v, perm, inv, gather ? xs : nullptr,
+                                      gather ? vs : nullptr, invnorm, hist, hdr, st);
+  return launch_sort<float>(D, buckets, x, v, perm, inv, gather ? xs : nullptr,
+                            gather ? vs : nullptr, invnorm, hist, hdr, st);
+}
+
+lsh_status lsh_attn_forward(const lsh_attn_desc* desc, const void* x, const void* v,
+                            const void* R, const int32_t* buckets, void* out, float* lse,
+                            void* ws, size_t ws_bytes, void* stream) {
+  return lsh_attn_forward_profiled(desc, x, v, R, buckets, out, lse, ws, ws_bytes, stream,
+                                   nullptr);
+}
+
+lsh_status lsh_attn_forward_profiled(const lsh_attn_desc* desc, const void* x, const void* v,
+                                     const void* R, const int32_t* buckets, void* out, float* lse,
+                                     void* ws, size_t ws_bytes, void* stream,
+                                     void* const* events) {
+  Dims D;
+  Layout L;
+  lsh_status s = check_desc(desc, &D, true);
+  if (s != LSH_OK) return s;
+  if (!x || !v || !out || !lse || (!buckets && !R)) return LSH_ERR_INVALID_ARG;
+  if (!(aligned16(x) && aligned16(v) && aligned16(out))) return LSH_ERR_INVALID_ARG;
+  if ((s = check_ws(D, ws, ws_bytes, &L)) != LSH_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = reset_header(ws, st)) != LSH_OK) return s;
+  return D.dtype == LSH_BF16
+             ? forward_typed<__nv_bfloat16>(D, L, x, v, R, buckets, out, lse, ws, st, events)
+             : forward_typed<float>(D, L, x, v, R, buckets, out, lse, ws, st, events);
+}
+
+lsh_status lsh_attn_get_diag(const void* ws, void* stream, lsh_attn_diag* diag) {
+  if (!ws || !diag) return LSH_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LSH_ERR_CUDA;
+  WsHeader h;
+  if (cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return LSH_ERR_CUDA;
+  diag->status = h.status;
+  diag->hash_refined = h.hash_refined;
+  diag->bad_bucket_ids = h.bad_bucket_ids;
+  diag->reserved = 0;
+  return LSH_OK;
+}
+
+lsh_status lsh_attn_get_device_status(const void* ws, void* stream) {
+  lsh_attn_diag d;
+  lsh_status s = lsh_attn_get_diag(ws, stream, &d);
+  if (s != LSH_OK) return s;
+  return static_cast<lsh_status>(d.status);
+}
+
+}  // extern "C"

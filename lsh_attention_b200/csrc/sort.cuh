@@ -1,0 +1,207 @@
+// Stable counting sort of every (batch, head, round) by bucket, then position,
+// fused with the gather of x and v rows into sorted order.
+//
+// "Reformer summary" (ttnews.xyz), §局部敏感哈希注意力: order the tokens by
+// bucket, and inside a bucket by position. Positions are already in order, so
+// slot(i) = #{j : b_j < b_i} + #{j < i : b_j = b_i}. Three kernels compute it
+// without a global sort:
+//   k_sort_hist     per-(segment, tile) bucket histograms, warp-aggregated
+//   k_sort_scan     exclusive scan of each segment's [bucket][tile] counts
+//   k_sort_scatter  per-warp counts inside the tile, stable ranks from
+//                   __match_any_sync, perm/inv writes, and the row gather
+// A segment is one (batch, head, round); a tile is kSortWarps(nb) warps of
+// kSortSub tokens each.
+#pragma once
+
+#include "common.cuh"
+
+namespace lsh {
+
+constexpr int kSortSub = 256;  // tokens per warp sub-range
+
+// Warps per tile: per-warp counters take warps * nb * 4 bytes of shared memory.
+__host__ __device__ inline int sort_warps(int nb) {
+  int w = 16384 / nb;
+  return w < 1 ? 1 : (w > 16 ? 16 : w);
+}
+__host__ __device__ inline int sort_tile(int nb) { return sort_warps(nb) * kSortSub; }
+
+__device__ __forceinline__ int clamp_bucket(int b, int nb) { return b < 0 ? 0 : (b >= nb ? nb - 1 : b); }
+
+// grid (tiles, segments), block 256. hist [seg][nb][tiles].
+__global__ void __launch_bounds__(256)
+    k_sort_hist(const int32_t* __restrict__ buckets, int n, int nb, int tile, int tiles,
+                int32_t* __restrict__ hist, WsHeader* hdr) {
+  extern __shared__ int32_t cnt[];
+  const int seg = blockIdx.y, tl = blockIdx.x;
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) cnt[b] = 0;
+  __syncthreads();
+  const int start = tl * tile, end = min(n, start + tile);
+  const int32_t* bk = buckets + (int64_t)seg * n;
+  const int lane = threadIdx.x & 31;
+  for (int base = start; base < end; base += blockDim.x) {
+    const int t = base + threadIdx.x;
+    int b = -1;
+    if (t < end) {
+      const int raw = bk[t];
+      b = clamp_bucket(raw, nb);
+      if (b != raw) {
+        atomicAdd(&hdr->bad_bucket_ids, 1u);
+        record_status(hdr, 6u /* LSH_ERR_DEVICE */);
+      }
+    }
+    const uint32_t peers = __match_any_sync(0xffffffffu, b);
+    if (b >= 0 && lane == __ffs(peers) - 1) atomicAdd(&cnt[b], __popc(peers));
+  }
+  __syncthreads();
+  int32_t* h = hist + (int64_t)seg * nb * tiles + tl;
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) h[(int64_t)b * tiles] = cnt[b];
+}
+
+// grid (segments), block 1024: in-place exclusive scan of len ints per segment.
+__global__ void __launch_bounds__(1024) k_sort_scan(int32_t* __restrict__ hist, int len) {
+  __shared__ int32_t wsum[32];
+  int32_t* h = hist + (int64_t)blockIdx.x * len;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t carry = 0;
+  for (int base = 0; base < len; base += 4 * 1024) {
+    const int i0 = base + 4 * threadIdx.x;
+    int32_t v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = (i0 + k < len) ? h[i0 + k] : 0;
+    const int32_t local = v[0] + v[1] + v[2] + v[3];
+    int32_t incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int32_t s = wsum[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += y;
+      }
+      wsum[lane] = s;  // inclusive over warps
+    }
+    __syncthreads();
+    int32_t run = carry + (warp > 0 ? wsum[warp - 1] : 0) + incl - local;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (i0 + k < len) h[i0 + k] = run;
+      run += v[k];
+    }
+    carry += wsum[31];
+    __syncthreads();
+  }
+}
+
+// Copy 32 rows (one per lane's token) of x and v into sorted order and write
+// each row's inverse key norm. Lane L holds the slot of token t0 + L.
+template <typename T>
+__device__ __forceinline__ void gather_rows(const T* __restrict__ xg, const T* __restrict__ vg,
+                                            int t0, int valid_count, int slot_mine, int d,
+                                            T* __restrict__ xs, T* __restrict__ vs,
+                                            float* __restrict__ invnorm) {
+  const int lane = threadIdx.x & 31;
+  const int cpr = d * (int)sizeof(T) / 16;  // 16-byte chunks per row (8..32)
+  const int rpp = 32 / cpr > 0 ? 32 / cpr : 1;  // rows per pass
+  const int lanes_per_row = cpr < 32 ? cpr : 32;
+  const int iters_per_row = cpr / lanes_per_row;  // 1, or 2 for 512-byte rows
+#pragma unroll 4
+  for (int r0 = 0; r0 < 32; r0 += rpp) {
+    const int ri = r0 + lane / lanes_per_row;
+    const int c = lane % lanes_per_row;
+    const int slot = __shfl_sync(0xffffffffu, slot_mine, ri & 31);
+    const bool ok = ri < valid_count;
+    float ss = 0.f;
+    if (ok) {
+      const uint4* xr = reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + ri) * d);
+      const uint4* vr = reinterpret_cast<const uint4*>(vg + (int64_t)(t0 + ri) * d);
+      uint4* xo = reinterpret_cast<uint4*>(xs + (int64_t)slot * d);
+      uint4* vo = reinterpret_cast<uint4*>(vs + (int64_t)slot * d);
+      for (int it = 0; it < iters_per_row; ++it) {
+        const int cc = c + it * lanes_per_row;
+        const uint4 a = __ldg(xr + cc);
+        const uint4 b = __ldg(vr + cc);
+        xo[cc] = a;
+        vo[cc] = b;
+        float f[Vec16<T>::N];
+        Vec16<T>::unpack(a, f);
+#pragma unroll
+        for (int k = 0; k < Vec16<T>::N; ++k) ss = fmaf(f[k], f[k], ss);
+      }
+    }
+    for (int o = lanes_per_row / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (ok && c == 0) invnorm[slot] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+  }
+}
+
+// grid (tiles, segments), block sort_warps(nb) * 32.
+// hist: scanned offsets [seg][nb][tiles]. perm, inv, invnorm: [seg][n];
+// xs, vs: [seg][n][d] (skipped when xs == nullptr). x, v: [BH][n][d].
+template <typename T>
+__global__ void __launch_bounds__(512)
+    k_sort_scatter(const int32_t* __restrict__ buckets, const int32_t* __restrict__ hist,
+                   const T* __restrict__ x, const T* __restrict__ v, int32_t* __restrict__ perm,
+                   int32_t* __restrict__ inv, T* __restrict__ xs, T* __restrict__ vs,
+                   float* __restrict__ invnorm, int n, int d, int nb, int rounds, int tiles) {
+  extern __shared__ int32_t base[];  // [warps][nb]
+  const int seg = blockIdx.y, tl = blockIdx.x;
+  const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < nw * nb; i += blockDim.x) base[i] = 0;
+  __syncthreads();
+
+  const int tile = nw * kSortSub;
+  const int wstart = tl * tile + warp * kSortSub;
+  const int wend = min(n, wstart + kSortSub);
+  const int32_t* bk = buckets + (int64_t)seg * n;
+  int32_t* mybase = base + warp * nb;
+
+  // 1) per-warp counts of its sub-range
+  for (int s0 = wstart; s0 < wend; s0 += 32) {
+    const int t = s0 + lane;
+    const int b = t < wend ? clamp_bucket(bk[t], nb) : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, b);
+    if (b >= 0 && lane == __ffs(peers) - 1) mybase[b] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // 2) exclusive scan over warps, seeded with the tile's offset for the bucket
+  const int32_t* h = hist + (int64_t)seg * nb * tiles + tl;
+  for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+    int32_t run = h[(int64_t)b * tiles];
+    for (int w = 0; w < nw; ++w) {
+      const int32_t c = base[w * nb + b];
+      base[w * nb + b] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  // 3) stable ranks, perm / inv, and the gather
+  const int64_t bh = seg / rounds;
+  const T* xg = x + bh * (int64_t)n * d;
+  const T* vg = v + bh * (int64_t)n * d;
+  const int64_t so = (int64_t)seg * n;
+  for (int s0 = wstart; s0 < wend; s0 += 32) {
+    const int t = s0 + lane;
+    const int b = t < wend ? clamp_bucket(bk[t], nb) : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, b);
+    int slot = 0;
+    if (b >= 0) slot = mybase[b] + __popc(peers & lanemask_lt());
+    __syncwarp();
+    if (b >= 0 && lane == __ffs(peers) - 1) mybase[b] += __popc(peers);
+    __syncwarp();
+    if (b >= 0) {
+      perm[so + slot] = t;
+      inv[so + t] = slot;
+    }
+    if (xs != nullptr)
+      gather_rows<T>(xg, vg, s0, wend - s0, slot, d, xs + so * d, vs + so * d, invnorm + so);
+  }
+}
+
+}  // namespace lsh
