@@ -1,0 +1,408 @@
+// Angular LSH hash for bf16 inputs on the 5th-generation tensor cores.
+//
+// "Reformer summary" (ttnews.xyz), §局部敏感哈希 and §多輪LSH哈希: for every
+// round r, p = x R_r (R_r of size [d, b/2]) and h(x) = argmax([p ; -p]).
+//
+// Design (persistent, warp-specialised, one CTA per SM):
+//   * the rotations of a group of rounds stay resident in shared memory
+//     (transposed to K-major by k_hash_prep, loaded once by TMA);
+//   * warp 0 streams 128-token tiles of x with TMA (double-buffered);
+//   * warp 1 issues tcgen05.mma (M = 128 tokens, N <= 256 columns, K = d)
+//     into one of two TMEM accumulators, so the next unit's MMA overlaps the
+//     epilogue of the current one;
+//   * warps 2..9 read the fp32 projections with tcgen05.ld and keep, per
+//     token, the largest and second largest |p_j|, the argmax and its sign.
+// Exactness: the fp32 accumulation of d bf16 products is within
+// d * 2^-23 * sum_k |x_k R_kj| <= d * 2^-23 * ||x|| ||R_j|| of the exact sum,
+// whatever the order or rounding of the additions. When the top two |p| are
+// closer than four times that bound (kTieFactor), the token is queued and
+// k_hash_refine re-decides it in fp64 in the sequential order of the
+// definition, so the bucket equals the exact argmax bit for bit.
+#pragma once
+
+#include "common.cuh"
+#include "hash_exact.cuh"
+#include "sm100.cuh"
+
+namespace lsh {
+
+constexpr int kHashTile = 128;       // tokens per tile (MMA M)
+constexpr int kHashMaxN = 256;       // columns per MMA (N)
+constexpr int kHashWarps = 10;       // 0: TMA, 1: MMA, 2..9: epilogue
+constexpr float kTieFactor = 4.0f;   // margin threshold / accumulation error bound
+constexpr int kHashSmemBudget = 227 * 1024;
+
+struct HashTcPlan {
+  int d, kh;        // head dim and its 64-element halves
+  int half, nc, ch; // nb/2, MMA N, column chunks per round
+  int group;        // rounds resident per CTA
+  int groups;       // ceil(rounds / group)
+  int tmem_cols;    // per accumulator buffer (power of two >= 32)
+  size_t smem;      // dynamic shared memory
+  size_t x_bytes, r_bytes;
+};
+
+// Shared-memory plan; group == 0 when even one round's R does not fit.
+inline HashTcPlan hash_tc_plan(int d, int nb, int rounds) {
+  HashTcPlan p{};
+  p.d = d;
+  p.kh = d / 64;
+  p.half = nb / 2;
+  int nc = ((p.half + 15) / 16) * 16;
+  p.nc = nc > kHashMaxN ? kHashMaxN : nc;
+  p.ch = (p.half + p.nc - 1) / p.nc;
+  p.x_bytes = (size_t)2 * p.kh * kHashTile * 128;
+  const size_t per_round = (size_t)p.ch * p.kh * p.nc * 128;
+  const size_t misc = 1024 /* alignment */ + 8192 /* barriers, combine buffers */;
+  const size_t avail = kHashSmemBudget > (long)(p.x_bytes + misc)
+                           ? kHashSmemBudget - p.x_bytes - misc
+                           : 0;
+  int g = (int)(avail / per_round);
+  if (g > rounds) g = rounds;
+  p.group = g;
+  p.groups = g > 0 ? (rounds + g - 1) / g : 0;
+  p.r_bytes = per_round * (size_t)g;
+  int tc = 32;
+  while (tc < p.nc) tc <<= 1;
+  p.tmem_cols = tc;
+  p.smem = p.x_bytes + p.r_bytes + misc;
+  return p;
+}
+
+// ---------------------------------------------------------------------------
+// R [rounds][d][half] -> Rt [rounds][ch * nc][d]: K-major rows for the MMA's
+// B operand, each round padded with zero rows to whole chunks of nc. Also,
+// per round, an upper bound of max_j ||R_j|| (float bits in rnorm_bits[r],
+// zeroed before the launch).
+// grid (ceil(ch * nc / 128), rounds), block 128.
+__global__ void __launch_bounds__(128)
+    k_hash_prep(const __nv_bfloat16* __restrict__ R, __nv_bfloat16* __restrict__ Rt,
+                uint32_t* __restrict__ rnorm_bits, int d, int half, int rows_per_round) {
+  const int r = blockIdx.y;
+  const int j = blockIdx.x * 128 + threadIdx.x;
+  if (j >= rows_per_round) return;
+  __nv_bfloat16* dst = Rt + ((int64_t)r * rows_per_round + j) * d;
+  if (j >= half) {
+    for (int k = 0; k < d; ++k) dst[k] = __float2bfloat16_rn(0.f);
+    return;
+  }
+  const __nv_bfloat16* src = R + (int64_t)r * d * half + j;
+  double ss = 0.0;
+  for (int k = 0; k < d; ++k) {
+    const __nv_bfloat16 e = src[(int64_t)k * half];
+    dst[k] = e;
+    const double f = (double)__bfloat162float(e);
+    ss += f * f;
+  }
+  const float nrm = __double2float_ru(sqrt(ss));  // rounded up: an upper bound
+  atomicMax(rnorm_bits + r, __float_as_uint(nrm));  // non-negative floats order as uints
+}
+
+// ---------------------------------------------------------------------------
+// Exact fp64 re-decision of queued (token, round) pairs; one warp per entry.
+// entries: (bh * n + t) << 5 | r. Count in hdr->hash_refined.
+__global__ void __launch_bounds__(256)
+    k_hash_refine(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ R,
+                  const uint64_t* __restrict__ entries, int32_t* __restrict__ buckets, int n,
+                  int d, int nb, int rounds, const WsHeader* __restrict__ hdr) {
+  const int half = nb / 2;
+  const uint32_t count = hdr->hash_refined;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t e = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); e < count;
+       e += warps) {
+    const uint64_t code = entries[e];
+    const int r = (int)(code & 31);
+    const int64_t row = (int64_t)(code >> 5);  // bh * n + t
+    const int64_t bh = row / n;
+    const int t = (int)(row % n);
+    const __nv_bfloat16* xr = x + row * d;
+    const __nv_bfloat16* Rr = R + (int64_t)r * d * half;
+    double bv = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int j0 = 0; j0 < half; j0 += 32 * 8) {
+      double acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+      for (int k = 0; k < d; ++k) {
+        const double xk = (double)__bfloat162float(xr[k]);
+        const __nv_bfloat16* Rk = Rr + (int64_t)k * half;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = j0 + i * 32 + lane;
+          if (j < half) acc[i] = fma(xk, (double)__bfloat162float(Rk[j]), acc[i]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j = j0 + i * 32 + lane;
+        if (j < half) {
+          argmax_update(acc[i], j, bv, bi);
+          argmax_update(-acc[i], half + j, bv, bi);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      argmax_update(ov, oi, bv, bi);
+    }
+    if (lane == 0) buckets[(bh * rounds + r) * n + t] = bi;
+  }
+}
+
+// ---------------------------------------------------------------------------
+struct HashTcArgs {
+  int32_t* buckets;   // [BH][rounds][n]
+  uint64_t* refine;   // queue of near-tie entries
+  WsHeader* hdr;      // counters; rnorm bits in hdr->pad[0..rounds)
+  int n, nb, rounds, tiles_per_seq, tiles, ctas_per_group;
+};
+
+// Running top-2 of |p| with the argmax and its signed value.
+struct Top2 {
+  float m1, m2, sv;
+  int idx;
+  __device__ __forceinline__ void reset() {
+    m1 = 0.f;
+    m2 = 0.f;
+    sv = 0.f;
+    idx = 0;
+  }
+  __device__ __forceinline__ void add(float v, int j) {
+    const float a = fabsf(v);
+    const bool gt = a > m1;
+    m2 = gt ? m1 : fmaxf(m2, a);
+    idx = gt ? j : idx;
+    sv = gt ? v : sv;
+    m1 = gt ? a : m1;
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kHashWarps * 32, 1)
+    k_hash_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmr,
+              HashTcArgs a, HashTcPlan p) {
+  using namespace sm100;
+  constexpr int KH = D / 64;
+  constexpr uint32_t XBOX = kHashTile * 128;  // bytes of one 64-column box of x
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* xbuf = base;                   // [2][KH][128 rows][128 B]
+  unsigned char* rbuf = base + p.x_bytes;       // [group][ch][KH][nc rows][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rbuf + p.r_bytes);
+  uint64_t* r_full = bars + 0;
+  uint64_t* x_full = bars + 1;     // [2]
+  uint64_t* x_empty = bars + 3;    // [2]
+  uint64_t* acc_full = bars + 5;   // [2]
+  uint64_t* acc_empty = bars + 7;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
+  float4* comb = reinterpret_cast<float4*>(bars + 16);  // [2][4][32]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.x / a.ctas_per_group;
+  const int li = blockIdx.x % a.ctas_per_group;
+  const int r0 = g * p.group;
+  const int gr = min(p.group, a.rounds - r0);  // rounds in this group
+
+  if (threadIdx.x == 0) {
+    mbar_init(r_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(x_full + i, 1);
+      mbar_init(x_empty + i, 1 + 4);  // MMA commit + 4 norm-reading warps
+      mbar_init(acc_full + i, 1);
+      mbar_init(acc_empty + i, 8);    // 8 epilogue warps
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 2 * p.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&]() {
+    record_status(a.hdr, 5u /* LSH_ERR_TIMEOUT */);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmx);
+      prefetch_tensormap(&tmr);
+      mbar_expect_tx(r_full, (uint32_t)((size_t)gr * p.ch * KH * p.nc * 128));
+      for (int rl = 0; rl < gr; ++rl)
+        for (int c = 0; c < p.ch; ++c)
+          for (int kh = 0; kh < KH; ++kh) {
+            unsigned char* dst = rbuf + ((size_t)(rl * p.ch + c) * KH + kh) * p.nc * 128;
+            tma_load_2d(dst, &tmr, r_full, kh * 64, ((r0 + rl) * p.ch + c) * p.nc);
+          }
+      int it = 0;
+      for (int tile = li; tile < a.tiles; tile += a.ctas_per_group, ++it) {
+        const int xb = it & 1, xk = it >> 1;
+        if (xk > 0 && !mbar_wait(x_empty + xb, (xk - 1) & 1)) { fail(); break; }
+        if (*abort_flag) break;
+        const int bh = tile / a.tiles_per_seq;
+        const int row0 = bh * a.n + (tile % a.tiles_per_seq) * kHashTile;
+        mbar_expect_tx(x_full + xb, KH * XBOX);
+        for (int kh = 0; kh < KH; ++kh)
+          tma_load_2d(xbuf + (xb * KH + kh) * XBOX, &tmx, x_full + xb, kh * 64, row0);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kHashTile, p.nc);
+      bool ok = mbar_wait(r_full, 0);
+      if (!ok) fail();
+      int it = 0, u = 0;
+      for (int tile = li; ok && tile < a.tiles; tile += a.ctas_per_group, ++it) {
+        const int xb = it & 1, xk = it >> 1;
+        if (!mbar_wait(x_full + xb, xk & 1)) { fail(); break; }
+        tc_fence_after();
+        const uint32_t xaddr = smem_u32(xbuf + xb * KH * XBOX);
+        for (int rl = 0; rl < gr && ok; ++rl) {
+          for (int c = 0; c < p.ch; ++c, ++u) {
+            const int ab = u & 1, uk = u >> 1;
+            if (uk > 0 && !mbar_wait(acc_empty + ab, (uk - 1) & 1)) { fail(); ok = false; break; }
+            if (*abort_flag) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t raddr =
+                smem_u32(rbuf + (size_t)(rl * p.ch + c) * KH * p.nc * 128);
+            const uint32_t d_tmem = tmem + ab * p.tmem_cols;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const int kh = kk >> 2, ks = kk & 3;
+              const uint64_t adesc = desc_kmajor_sw128(xaddr + kh * XBOX + ks * 32);
+              const uint64_t bdesc = desc_kmajor_sw128(raddr + kh * p.nc * 128 + ks * 32);
+              mma_bf16_ss(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(acc_full + ab);
+          }
+        }
+        mma_commit(x_empty + xb);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;
+    const int q = warp & 3;       // TMEM lane quadrant this warp may access
+    const int h = e >> 2;         // column-batch parity handled by this warp
+    const int row = q * 32 + lane;
+    const uint32_t tlane = (uint32_t)(q * 32) << 16;
+    const float* rnorm = reinterpret_cast<const float*>(a.hdr->pad);
+    const int nbatch = p.nc / 16;
+    int it = 0, u = 0, rc = 0;
+    for (int tile = li; tile < a.tiles; tile += a.ctas_per_group, ++it) {
+      const int xb = it & 1, xk = it >> 1;
+      const int bh = tile / a.tiles_per_seq;
+      const int t = (tile % a.tiles_per_seq) * kHashTile + row;
+      // Failures set abort_flag before the next named barrier, so both warps
+      // of a quadrant leave the loop after the same barrier.
+      bool ok = true;
+      float xnorm = 0.f;
+      if (h == 0) {
+        if (!mbar_wait(x_full + xb, xk & 1)) {
+          fail();
+          ok = false;
+        } else {
+          // ||x_row|| from the swizzled tile: 16-byte chunk c of a row sits at
+          // slot c ^ (row % 8) of its 128-byte line.
+          float ss = 0.f;
+#pragma unroll
+          for (int kh = 0; kh < KH; ++kh) {
+            const unsigned char* line = xbuf + (xb * KH + kh) * XBOX + row * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 v = *reinterpret_cast<const uint4*>(line + ((c ^ (row & 7)) << 4));
+              float f[8];
+              Vec16<__nv_bfloat16>::unpack(v, f);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) ss = fmaf(f[k], f[k], ss);
+            }
+          }
+          xnorm = sqrtf(ss) * 1.0001f;  // covers the fp32 rounding of the norm
+          __syncwarp();
+          if (lane == 0) mbar_arrive(x_empty + xb);
+        }
+      }
+      bool stop = false;
+      for (int rl = 0; rl < gr; ++rl, ++rc) {
+        Top2 st;
+        st.reset();
+        for (int c = 0; ok && c < p.ch; ++c, ++u) {
+          const int ab = u & 1, uk = u >> 1;
+          if (!mbar_wait(acc_full + ab, uk & 1)) {
+            fail();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tbase = tmem + tlane + ab * p.tmem_cols;
+          for (int b = h; b < nbatch; b += 2) {
+            uint32_t v[16];
+            tmem_ld16(tbase + b * 16, v);
+            tmem_wait_ld();
+            const int j0 = c * p.nc + b * 16;
+            if (j0 + 16 <= p.half) {
+#pragma unroll
+              for (int k = 0; k < 16; ++k) st.add(__uint_as_float(v[k]), j0 + k);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+                if (j0 + k < p.half) st.add(__uint_as_float(v[k]), j0 + k);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty + ab);
+        }
+        // combine the two warps of this quadrant, then decide
+        float4* slot = comb + ((rc & 1) * 4 + q) * 32 + lane;
+        if (h == 1) *slot = make_float4(st.m1, st.m2, __int_as_float(st.idx), st.sv);
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+        stop = *abort_flag != 0;
+        if (stop) break;
+        if (h == 0) {
+          const float4 o = *slot;
+          const int oidx = __float_as_int(o.z);
+          float m1 = st.m1, m2, sv = st.sv;
+          int idx = st.idx;
+          if (o.x > st.m1 || (o.x == st.m1 && oidx < st.idx)) {
+            m2 = fmaxf(fmaxf(o.y, st.m2), st.m1);
+            m1 = o.x;
+            idx = oidx;
+            sv = o.w;
+          } else {
+            m2 = fmaxf(fmaxf(o.y, st.m2), o.x);
+          }
+          if (t < a.n) {
+            const int r = r0 + rl;
+            const float tau = kTieFactor * (float)D * 1.1920929e-7f * xnorm * rnorm[r];
+            const int bucket = idx + (sv < 0.f ? p.half : 0);
+            const int64_t at = ((int64_t)bh * a.rounds + r) * a.n + t;
+            a.buckets[at] = bucket;
+            if (!(m1 - m2 > tau)) {
+              const uint32_t k = atomicAdd(&a.hdr->hash_refined, 1u);
+              a.refine[k] = ((uint64_t)((int64_t)bh * a.n + t) << 5) | (uint64_t)r;
+            }
+          }
+        }
+      }
+      if (stop) break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * p.tmem_cols);
+  }
+}
+
+}  // namespace lsh

@@ -9,15 +9,17 @@
 #include "attn_simt.cuh"
 #include "common.cuh"
 #include "hash_exact.cuh"
+#include "hash_tc.cuh"
 #include "merge.cuh"
 #include "sort.cuh"
+#include "tma_host.cuh"
 
 namespace {
 
 using namespace lsh;
 
 struct Layout {
-  size_t header, buckets, perm, inv, invnorm, lse_s, hist, xs, vs, out_s, total;
+  size_t header, buckets, perm, inv, invnorm, lse_s, hist, xs, vs, out_s, rt, refine, total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -81,6 +83,9 @@ Layout layout_of(const Dims& D) {
   L.xs = take(sn * D.d * D.esize);
   L.vs = take(sn * D.d * D.esize);
   L.out_s = take(sn * D.d * 4);
+  const HashTcPlan hp = hash_tc_plan(D.d, D.nb, D.rounds);
+  L.rt = take((size_t)D.rounds * hp.ch * hp.nc * D.d * 2);  // R transposed (bf16 hash)
+  L.refine = take(sn * 8);                             // near-tie queue of the bf16 hash
   L.total = off;
   return L;
 }
@@ -107,20 +112,88 @@ lsh_status reset_header(void* ws, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- launches
-template <typename T>
-lsh_status launch_hash(const Dims& D, const void* x, const void* R, int32_t* buckets,
-                       cudaStream_t st) {
-  const int xstride = D.d + (sizeof(T) == 4 ? 1 : 2);
-  const size_t smem = sizeof(double) * D.d * kHashExactCols +
-                      sizeof(T) * (size_t)kHashExactTokens * xstride;
-  auto kern = k_hash_exact<T>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return LSH_ERR_CUDA;
+lsh_status launch_hash_exact(const Dims& D, const void* x, const void* R, int32_t* buckets,
+                             cudaStream_t st, bool bf16) {
+  const int esz = bf16 ? 2 : 4;
+  const int xstride = D.d + (esz == 4 ? 1 : 2);
+  const size_t smem =
+      sizeof(double) * D.d * kHashExactCols + (size_t)esz * kHashExactTokens * xstride;
   dim3 grid((D.n + kHashExactTokens - 1) / kHashExactTokens, (unsigned)D.BH, D.rounds);
-  kern<<<grid, kHashExactTokens, smem, st>>>(static_cast<const T*>(x), static_cast<const T*>(R),
-                                              buckets, D.n, D.d, D.nb, D.rounds);
+  if (bf16) {
+    auto kern = k_hash_exact<__nv_bfloat16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, kHashExactTokens, smem, st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                static_cast<const __nv_bfloat16*>(R), buckets,
+                                                D.n, D.d, D.nb, D.rounds);
+  } else {
+    auto kern = k_hash_exact<float>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, kHashExactTokens, smem, st>>>(static_cast<const float*>(x),
+                                                static_cast<const float*>(R), buckets, D.n, D.d,
+                                                D.nb, D.rounds);
+  }
   return last_cuda();
+}
+
+// bf16: tcgen05 projection + top-2 screen, fp64 re-decision of near ties.
+lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const void* R,
+                          int32_t* buckets, void* ws, cudaStream_t st) {
+  const HashTcPlan p = hash_tc_plan(D.d, D.nb, D.rounds);
+  if (p.group == 0) return launch_hash_exact(D, x, R, buckets, st, true);
+  WsHeader* hdr = at<WsHeader>(ws, L.header);
+  __nv_bfloat16* rt = at<__nv_bfloat16>(ws, L.rt);
+  uint64_t* refine = at<uint64_t>(ws, L.refine);
+  const int rows_per_round = p.ch * p.nc;
+  dim3 pg((rows_per_round + 127) / 128, D.rounds);
+  k_hash_prep<<<pg, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(R), rt, hdr->pad, D.d, p.half,
+                                  rows_per_round);
+  CUtensorMap tmx, tmr;
+  if (!make_tmap_bf16_2d(&tmx, x, D.d, (uint64_t)D.BH * D.n, (uint64_t)D.d * 2, 64, kHashTile) ||
+      !make_tmap_bf16_2d(&tmr, rt, D.d, (uint64_t)D.rounds * rows_per_round, (uint64_t)D.d * 2, 64,
+                         p.nc))
+    return LSH_ERR_CUDA;
+  HashTcArgs a;
+  a.buckets = buckets;
+  a.refine = refine;
+  a.hdr = hdr;
+  a.n = D.n;
+  a.nb = D.nb;
+  a.rounds = D.rounds;
+  a.tiles_per_seq = (D.n + kHashTile - 1) / kHashTile;
+  a.tiles = (int)(D.BH * a.tiles_per_seq);
+  const int sms = sm_count();
+  int per = sms / p.groups;
+  if (per < 1) per = 1;
+  if (per > a.tiles) per = a.tiles;
+  a.ctas_per_group = per;
+  const unsigned grid = (unsigned)(per * p.groups);
+  if (D.d == 64) {
+    auto kern = k_hash_tc<64>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, kHashWarps * 32, p.smem, st>>>(tmx, tmr, a, p);
+  } else {
+    auto kern = k_hash_tc<128>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, kHashWarps * 32, p.smem, st>>>(tmx, tmr, a, p);
+  }
+  k_hash_refine<<<2 * sms, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+                                         static_cast<const __nv_bfloat16*>(R), refine, buckets,
+                                         D.n, D.d, D.nb, D.rounds, hdr);
+  return last_cuda();
+}
+
+lsh_status launch_hash(const Dims& D, const Layout& L, const void* x, const void* R,
+                       int32_t* buckets, void* ws, cudaStream_t st) {
+  if (D.dtype == LSH_BF16) return launch_hash_tc(D, L, x, R, buckets, ws, st);
+  return launch_hash_exact(D, x, R, buckets, st, false);
 }
 
 template <typename T>
@@ -194,7 +267,7 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
   if ((s = mark(ev, 0, st)) != LSH_OK) return s;
   if (!buckets) {
     int32_t* bk = at<int32_t>(ws, L.buckets);
-    if ((s = launch_hash<T>(D, x, R, bk, st)) != LSH_OK) return s;
+    if ((s = launch_hash(D, L, x, R, bk, ws, st)) != LSH_OK) return s;
     buckets = bk;
   }
   if ((s = mark(ev, 1, st)) != LSH_OK) return s;
@@ -253,11 +326,11 @@ lsh_status lsh_attn_hash(const lsh_attn_desc* desc, const void* x, const void* R
   lsh_status s = check_desc(desc, &D, false);
   if (s != LSH_OK) return s;
   if (!x || !R || !buckets) return LSH_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(R)) return LSH_ERR_INVALID_ARG;
   if ((s = check_ws(D, ws, ws_bytes, &L)) != LSH_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = reset_header(ws, st)) != LSH_OK) return s;
-  return D.dtype == LSH_BF16 ? launch_hash<__nv_bfloat16>(D, x, R, buckets, st)
-                             : launch_hash<float>(D, x, R, buckets, st);
+  return launch_hash(D, L, x, R, buckets, ws, st);
 }
 
 lsh_status lsh_attn_sort(const lsh_attn_desc* desc, const int32_t* buckets, const void* x,
@@ -303,6 +376,7 @@ lsh_status lsh_attn_forward_profiled(const lsh_attn_desc* desc, const void* x, c
   if (s != LSH_OK) return s;
   if (!x || !v || !out || !lse || (!buckets && !R)) return LSH_ERR_INVALID_ARG;
   if (!(aligned16(x) && aligned16(v) && aligned16(out))) return LSH_ERR_INVALID_ARG;
+  if (!buckets && !aligned16(R)) return LSH_ERR_INVALID_ARG;
   if ((s = check_ws(D, ws, ws_bytes, &L)) != LSH_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = reset_header(ws, st)) != LSH_OK) return s;

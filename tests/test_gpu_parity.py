@@ -291,3 +291,47 @@ def test_host_errors_write_nothing():
     assert e.value.status == 2
     torch.cuda.synchronize()
     assert (out == 7.0).all()
+
+
+# --------------------------------------------------------------------------
+# the tensor-core hash on exact ties and its fp64 re-decision queue
+@pytest.mark.parametrize("d,nb", [(64, 16), (128, 1024), (64, 2), (64, 192)])
+def test_hash_exact_ties_bit_exact(d, nb):
+    """Rows built to tie exactly (zero rows, basis vectors against duplicated
+    and negated columns of R) must take the first index of [xR ; -xR]."""
+    w = I.Workload("ties", 1, 1, 512, d, nb, 64, 2, True, "bf16")
+    x, _ = I.make_qkv(w)
+    R = I.make_rotations(w)
+    half = nb // 2
+    if half >= 4:
+        R[:, :, 1] = R[:, :, 0]    # duplicate column: p_1 == p_0
+        R[:, :, 3] = -R[:, :, 2]   # negated column: p_3 == -p_2
+    x[0, 0, :16] = 0                                       # all projections zero
+    for i in range(16, 48):
+        x[0, 0, i] = 0
+        x[0, 0, i, i % d] = 1.0 if i % 2 else -2.0         # basis vectors
+    ref, margin = oracle.hash_all(x, R)
+    xg, Rg = to_gpu(x, R)
+    desc = lb.make_desc(1, 1, 512, d, nb, 64, 2, True, torch.bfloat16)
+    ws = lb.workspace(desc, xg.device)
+    got = lb.lsh_attn_hash(xg, Rg, nb, ws=ws).cpu().numpy()
+    np.testing.assert_array_equal(got, ref)
+    diag = lb.lsh_attn_get_diag(ws)
+    assert diag["status"] == 0
+    assert diag["hash_refined"] >= 16  # at least the zero rows went through fp64
+
+
+def test_hash_refine_count_is_small():
+    w = I.LONG_64K
+    x, _ = I.make_qkv(w)
+    R = I.make_rotations(w)
+    xg, Rg = to_gpu(x, R)
+    desc = lb.make_desc(w.batch, w.heads, w.n, w.d, w.n_buckets, w.chunk, w.rounds, w.causal,
+                        torch.bfloat16)
+    ws = lb.workspace(desc, xg.device)
+    lb.lsh_attn_hash(xg, Rg, w.n_buckets, ws=ws)
+    diag = lb.lsh_attn_get_diag(ws)
+    total = w.batch * w.heads * w.n * w.rounds
+    print(f"{w.name}: {diag['hash_refined']} of {total} hashes re-decided in fp64")
+    assert diag["status"] == 0
+    assert 0 < diag["hash_refined"] < 0.02 * total
