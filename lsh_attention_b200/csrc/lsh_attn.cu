@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include "attn_simt.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 #include "hash_exact.cuh"
 #include "hash_tc.cuh"
@@ -241,6 +242,50 @@ lsh_status launch_attn_simt(const Dims& D, const void* xs, const void* vs, const
   return launch_attn_simt_q<T, DD, 16>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
 }
 
+// bf16, chunk 64: tcgen05 kernel on pairs of chunks.
+inline bool attn_tc_supported(const Dims& D) {
+  return D.dtype == LSH_BF16 && D.m == kAttnM && D.n % kAttnM == 0 &&
+         D.S * (int64_t)D.n < (int64_t(1) << 31);
+}
+
+lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
+                          const float* invnorm, float* out_s, float* lse_s, WsHeader* hdr,
+                          cudaStream_t st) {
+  CUtensorMap tmx, tmv;
+  const uint64_t rows = (uint64_t)D.S * D.n;
+  if (!make_tmap_bf16_2d(&tmx, xs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys) ||
+      !make_tmap_bf16_2d(&tmv, vs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys))
+    return LSH_ERR_CUDA;
+  AttnTcArgs a;
+  a.invnorm = invnorm;
+  a.perm = perm;
+  a.out_s = out_s;
+  a.lse_s = lse_s;
+  a.hdr = hdr;
+  a.n = D.n;
+  a.causal = D.causal;
+  a.pairs_per_seg = (D.n / kAttnM + 1) / 2;
+  a.pairs = D.S * a.pairs_per_seg;
+  const int64_t ctas_max = 2 * (int64_t)sm_count();
+  a.pairs_per_cta = (a.pairs + ctas_max - 1) / ctas_max;
+  const unsigned grid = (unsigned)((a.pairs + a.pairs_per_cta - 1) / a.pairs_per_cta);
+  const size_t smem = attn_tc_smem(D.d);
+  if (D.d == 64) {
+    auto kern = k_attn_tc<64>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, 128, smem, st>>>(tmx, tmv, a);
+  } else {
+    auto kern = k_attn_tc<128>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, 128, smem, st>>>(tmx, tmv, a);
+  }
+  return last_cuda();
+}
+
 template <typename T, int DD>
 lsh_status launch_merge(const Dims& D, const int32_t* inv, const float* lse_s, const float* out_s,
                         void* out, float* lse, cudaStream_t st) {
@@ -282,8 +327,11 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
                           hdr, st)) != LSH_OK)
     return s;
   if ((s = mark(ev, 2, st)) != LSH_OK) return s;
-  s = D.d == 64 ? launch_attn_simt<T, 64>(D, xs, vs, perm, invnorm, out_s, lse_s, st)
-                : launch_attn_simt<T, 128>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
+  if (attn_tc_supported(D))
+    s = launch_attn_tc(D, xs, vs, perm, invnorm, out_s, lse_s, hdr, st);
+  else
+    s = D.d == 64 ? launch_attn_simt<T, 64>(D, xs, vs, perm, invnorm, out_s, lse_s, st)
+                  : launch_attn_simt<T, 128>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
   if (s != LSH_OK) return s;
   if ((s = mark(ev, 3, st)) != LSH_OK) return s;
   s = D.d == 64 ? launch_merge<T, 64>(D, inv, lse_s, out_s, out, lse, st)
