@@ -1,27 +1,30 @@
 // Chunked shared-QK attention on the 5th-generation tensor cores (bf16 in,
-// fp32 accumulate), for chunks of m = 64 sorted slots.
+// fp32 accumulate), chunk m = 64, as a warp-specialised pipeline.
 //
 // "Reformer summary" (ttnews.xyz), §局部敏感哈希注意力 (chunks of m in the
 // sorted order), §共享QK中的自掩碼 (self-mask); "Reformer: LSH attention and
 // reversible layers" (dtcms.com), §二.1 (unit-length keys, 1/sqrt(d_k)).
 // A query in chunk c sees the keys of chunks c-1 and c.
 //
-// One work unit is a pair of chunks (c0, c0+1) of one (batch, head, round):
-// its 128 queries are slots [64 c0, 64 c0 + 128) and its 192-key window is
-// slots [64 (c0 - 1), 64 (c0 + 2)); the queries are rows 64..191 of the key
-// tile, so Q needs no load of its own. Per unit:
-//   TMA     sorted x and v rows of the window (2 x 192 rows), key norms and
-//           positions (bulk copies) -> shared memory
-//   MMA 1   S = Q K^T (M 128, N 192, K d) -> TMEM columns [0, 192)
-//   softmax thread i owns query row i: reads its 128 in-window logits with
-//           tcgen05.ld, applies 1/||k_j|| / sqrt(d), the causal mask and the
-//           -1e5 self logit, and writes P (bf16, zero outside the window)
-//           back to TMEM columns [0, 96) with tcgen05.st
-//   MMA 2   O = P V (A = P from TMEM, B = V, MN-major) -> TMEM [128, 128 + d)
-//   store   O / sum and lse, fp32, in slot order
-// X is re-loaded as soon as MMA 1 completes and V as soon as MMA 2 does, and
-// two CTAs share each SM (256 TMEM columns, < 114 KB shared memory each), so
-// one CTA's loads overlap the other's math.
+// Work unit: a pair of chunks (c0, c0+1) of one (batch, head, round). Its 128
+// queries are slots [64 c0, 64 c0 + 128) and its key window is slots
+// [64 (c0-1), 64 (c0+2)): the queries are rows 64..191 of the key tile.
+//
+// One persistent CTA per SM walks a contiguous range of units:
+//   warp 0      TMA: x tile, key norms and positions (stage s = unit & 1),
+//               then the v tile; each as soon as its stage is released
+//   warp 1      tcgen05.mma: S(u+1) = Q K^T into TMEM S[s], then O(u) = P V
+//               with P read from TMEM, so S of the next unit is ready when
+//               the softmax warps finish the current one
+//   warps 2..5  softmax, one query row per thread, one pass: logits in log2
+//               units are bounded by ||q|| log2(e) / sqrt(d) (keys have unit
+//               length), which serves as the stabiliser, so every probability
+//               is exp2(l - bound) <= 1 and is written to TMEM (bf16, over the
+//               dead S columns) as soon as it is computed; the row sum goes to
+//               the epilogue. A row whose only visible key is itself (the -1e5
+//               self logit) is flagged: its output is v of the query itself.
+//   warps 6..9  epilogue: O from TMEM, divided by the row sum, stored fp32
+// TMEM: S[0] = [0, 192), S[1] = [192, 384), O = [384, 384 + d).
 #pragma once
 
 #include "common.cuh"
@@ -31,316 +34,319 @@ namespace lsh {
 
 constexpr int kAttnM = 64;      // chunk length served by this kernel
 constexpr int kAttnKeys = 192;  // key window of a pair of chunks
-constexpr int kAttnTmemCols = 256;
+constexpr int kAttnWarps = 10;
+constexpr int kAttnStats = 4;   // row-sum slots between softmax and epilogue
+// Above this bound (log2 units) the stabiliser could push exp2 below the
+// normal range: those rows use their exact maximum instead.
+constexpr float kAttnBoundMax = 60.f;
 
 struct AttnTcArgs {
-  const float* invnorm;  // [S][n]
-  const int32_t* perm;   // [S][n]
-  float* out_s;          // [S][n][d] fp32, slot order
-  float* lse_s;          // [S][n]
+  const float* invnorm;        // [S][n] 1/||x|| of the sorted rows (0 for a zero row)
+  const int32_t* perm;         // [S][n] position of each slot
+  const __nv_bfloat16* vs;     // [S][n][d] sorted v rows (self-only rows copy theirs)
+  float* out_s;                // [S][n][d] fp32, slot order
+  float* lse_s;                // [S][n]
   WsHeader* hdr;
   int n, causal, pairs_per_seg;
-  int64_t pairs;         // S * pairs_per_seg
+  int64_t pairs;               // S * pairs_per_seg
   int64_t pairs_per_cta;
 };
-
-__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
-                                              uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(sm100::smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(sm100::smem_u32(bar))
-      : "memory");
-}
-
-// 32 lanes x 32 consecutive 32-bit TMEM columns.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem], kind::f16.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Shared-memory descriptor of an MN-major operand with the 128-byte swizzle:
-// 64-element MN blocks `lbo` bytes apart, 8-row K groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// P row of one query: 192 keys packed two per 32-bit column, zero outside the
-// 128 in-window keys starting at column WCOL; written to TMEM columns [0, 96).
-template <int WCOL>
-__device__ __forceinline__ void store_p_row(const float (&e)[128], uint32_t taddr) {
-#pragma unroll
-  for (int b = 0; b < 3; ++b) {
-    uint32_t pk[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const int i = b * 64 + 2 * k - WCOL;
-      const float e0 = (i >= 0 && i < 128) ? e[(i >= 0 && i < 128) ? i : 0] : 0.f;
-      const float e1 = (i + 1 >= 0 && i + 1 < 128) ? e[(i + 1 >= 0 && i + 1 < 128) ? i + 1 : 0] : 0.f;
-      pk[k] = pack_bf16x2(e0, e1);
-    }
-    tmem_st32(taddr + b * 32, pk);
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(128, 2)
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kAttnWarps * 32, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmv,
               AttnTcArgs a) {
   using namespace sm100;
   constexpr int KH = D / 64;
-  constexpr uint32_t BOX = kAttnKeys * 128;  // one 64-column box of 192 rows
-  constexpr uint32_t TILE = KH * BOX;        // x (or v) tile of the window
+  constexpr uint32_t BOX = kAttnKeys * 128;
+  constexpr uint32_t TILE = KH * BOX;
   constexpr float kLog2e = 1.4426950408889634f;
+  constexpr int kNoKey = 0x7fffffff;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* xt = base;            // [KH][192 rows][128 B]
-  unsigned char* vt = base + TILE;     // [KH][192 rows][128 B]
-  float* kinv = reinterpret_cast<float*>(base + 2 * TILE);  // [2][192]
+  unsigned char* xt = base;                                          // [2][KH][192][128 B]
+  unsigned char* vt = base + 2 * TILE;                               // [2][KH][192][128 B]
+  float* kinv = reinterpret_cast<float*>(base + 4 * TILE);           // [2][192]
   int32_t* kpos = reinterpret_cast<int32_t*>(kinv + 2 * kAttnKeys);  // [2][192]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(kpos + 2 * kAttnKeys);
-  uint64_t* x_full = bars + 0;
-  uint64_t* v_full = bars + 1;
-  uint64_t* s_done = bars + 2;
-  uint64_t* o_done = bars + 3;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  float2* ktab = reinterpret_cast<float2*>(kpos + 2 * kAttnKeys);    // [2][192] (scale, pos)
+  float* rstat = reinterpret_cast<float*>(ktab + 2 * kAttnKeys);     // [4][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(rstat + kAttnStats * 128);
+  uint64_t* xfull = bars + 0;    // [2] tx: x tile + metadata
+  uint64_t* xfree = bars + 2;    // [2] S MMA done + 4 softmax warps done with the metadata
+  uint64_t* vfull = bars + 4;    // [2]
+  uint64_t* vfree = bars + 6;    // [2] PV MMA done
+  uint64_t* sfull = bars + 8;    // [2] S MMA done
+  uint64_t* pready = bars + 10;  // [2] P written (4 softmax warps)
+  uint64_t* sfree = bars + 12;   // [2] PV MMA done with P
+  uint64_t* ofull = bars + 14;   // PV MMA done
+  uint64_t* ofree = bars + 15;   // 4 epilogue warps done reading O
+  uint64_t* statf = bars + 16;   // [4] row sums written (4 softmax warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t p_begin = blockIdx.x * a.pairs_per_cta;
-  const int64_t p_end = min(a.pairs, p_begin + a.pairs_per_cta);
-  if (p_begin >= p_end) return;  // uniform across the CTA
+  const int64_t u0 = blockIdx.x * a.pairs_per_cta;
+  const int64_t u1 = min(a.pairs, u0 + a.pairs_per_cta);
+  if (u0 >= u1) return;  // uniform across the CTA
+  const int nu = (int)(u1 - u0);
 
   if (tid == 0) {
-    mbar_init(x_full, 1);
-    mbar_init(v_full, 1);
-    mbar_init(s_done, 1);
-    mbar_init(o_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(xfull + i, 1);
+      mbar_init(xfree + i, 1 + 4);
+      mbar_init(vfull + i, 1);
+      mbar_init(vfree + i, 1);
+      mbar_init(sfull + i, 1);
+      mbar_init(pready + i, 4);
+      mbar_init(sfree + i, 1);
+    }
+    mbar_init(ofull, 1);
+    mbar_init(ofree, 4);
+    for (int i = 0; i < kAttnStats; ++i) mbar_init(statf + i, 4);
+    *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) tmem_alloc(tmem_slot, kAttnTmemCols);
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tm_s = tmem;        // S [0, 192), then P [0, 96)
-  const uint32_t tm_o = tmem + 128;  // O [128, 128 + D): S is dead by then
+  const uint32_t tm_o = tmem + 384;
 
-  // Issue the loads of x rows, key norms and positions (x_full) or of v rows
-  // (v_full) for unit p into meta buffer `mb`.
-  auto load_x = [&](int64_t p, int mb) {
-    const int64_t seg = p / a.pairs_per_seg;
-    const int c0 = (int)(p % a.pairs_per_seg) * 2;
-    const int k0 = (c0 - 1) * kAttnM;  // first key slot of the window (may be < 0)
-    const int lo = max(0, k0), hi = min(a.n, k0 + kAttnKeys);
-    const uint32_t mbytes = (uint32_t)(hi - lo) * 4;
-    mbar_expect_tx(x_full, TILE + 2 * mbytes);
-    const int row = (int)(seg * a.n) + k0;
-    for (int kh = 0; kh < KH; ++kh) tma_load_2d(xt + kh * BOX, &tmx, x_full, kh * 64, row);
-    bulk_copy_g2s(kinv + mb * kAttnKeys + (lo - k0), a.invnorm + seg * a.n + lo, mbytes, x_full);
-    bulk_copy_g2s(kpos + mb * kAttnKeys + (lo - k0), a.perm + seg * a.n + lo, mbytes, x_full);
+  auto fail = [&]() {
+    record_status(a.hdr, 5u /* LSH_ERR_TIMEOUT */);
+    *abort_flag = 1;
   };
-  auto load_v = [&](int64_t p) {
-    const int64_t seg = p / a.pairs_per_seg;
-    const int c0 = (int)(p % a.pairs_per_seg) * 2;
-    const int row = (int)(seg * a.n) + (c0 - 1) * kAttnM;
-    mbar_expect_tx(v_full, TILE);
-    for (int kh = 0; kh < KH; ++kh) tma_load_2d(vt + kh * BOX, &tmv, v_full, kh * 64, row);
-  };
+  auto unit_seg = [&](int i) { return (u0 + i) / a.pairs_per_seg; };
+  auto unit_c0 = [&](int i) { return (int)((u0 + i) % a.pairs_per_seg) * 2; };
 
-  if (tid == 0) {
-    prefetch_tensormap(&tmx);
-    prefetch_tensormap(&tmv);
-    load_x(p_begin, 0);
-    load_v(p_begin);
-  }
-
-  const uint32_t idesc_s = idesc_bf16_f32(128, kAttnKeys);
-  const uint32_t idesc_o = idesc_bf16_f32(128, D) | (1u << 16);  // B (= V) MN-major
-  const float qk_scale = 1.0f / sqrtf((float)D);
-  const int row = warp * 32 + lane;         // query row of the unit = TMEM lane
-  const int wcol = warp < 2 ? 0 : kAttnM;   // first in-window key column of this warp
-  const uint32_t tl = (uint32_t)(warp * 32) << 16;
-  bool ok = true;
-
-  int it = 0;
-  for (int64_t p = p_begin; p < p_end; ++p, ++it) {
-    const int mb = it & 1;
-    const uint32_t ph = it & 1;
-    const int64_t seg = p / a.pairs_per_seg;
-    const int c0 = (int)(p % a.pairs_per_seg) * 2;
-    const int k0 = (c0 - 1) * kAttnM;
-
-    // ---- MMA 1: S = Q K^T
-    if (tid == 0) {
-      if (mbar_wait(x_full, ph)) {
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmx);
+      prefetch_tensormap(&tmv);
+      bool ok = true;
+      for (int i = 0; ok && i < nu && !*abort_flag; ++i) {
+        const int s = i & 1, k = i >> 1;
+        const int64_t seg = unit_seg(i);
+        const int k0 = (unit_c0(i) - 1) * kAttnM;  // first key slot (may be < 0)
+        const int row = (int)(seg * a.n) + k0;
+        if (k > 0 && !mbar_wait(xfree + s, (k - 1) & 1)) { ok = false; break; }
+        const int lo = max(0, k0), hi = min(a.n, k0 + kAttnKeys);
+        const uint32_t mbytes = (uint32_t)(hi - lo) * 4;
+        mbar_expect_tx(xfull + s, TILE + 2 * mbytes);
+        for (int kh = 0; kh < KH; ++kh)
+          tma_load_2d(xt + s * TILE + kh * BOX, &tmx, xfull + s, kh * 64, row);
+        bulk_copy_g2s(kinv + s * kAttnKeys + (lo - k0), a.invnorm + seg * a.n + lo, mbytes,
+                      xfull + s);
+        bulk_copy_g2s(kpos + s * kAttnKeys + (lo - k0), a.perm + seg * a.n + lo, mbytes,
+                      xfull + s);
+        if (k > 0 && !mbar_wait(vfree + s, (k - 1) & 1)) { ok = false; break; }
+        mbar_expect_tx(vfull + s, TILE);
+        for (int kh = 0; kh < KH; ++kh)
+          tma_load_2d(vt + s * TILE + kh * BOX, &tmv, vfull + s, kh * 64, row);
+      }
+      if (!ok) fail();
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, kAttnKeys);
+      const uint32_t idesc_o = idesc_bf16_f32(128, D) | (1u << 16);  // B = V, MN-major
+      auto issue_s = [&](int i) {
+        const int s = i & 1, k = i >> 1;
+        if (!mbar_wait(xfull + s, k & 1)) return false;
+        if (k > 0 && !mbar_wait(sfree + s, (k - 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t xa = smem_u32(xt);
+        const uint32_t xa = smem_u32(xt + s * TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int kh = kk >> 2, ks = kk & 3;
           const uint64_t ad = desc_kmajor_sw128(xa + kh * BOX + kAttnM * 128 + ks * 32);
           const uint64_t bd = desc_kmajor_sw128(xa + kh * BOX + ks * 32);
-          mma_bf16_ss(tm_s, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + s * 192, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_done);
-      } else {
-        ok = false;
-      }
-    }
-    if (!__syncthreads_and(ok)) break;
-    if (!mbar_wait(s_done, ph)) ok = false;
-    tc_fence_after();
-    // x tile is free again: prefetch the next unit's rows and metadata
-    if (tid == 0 && ok && p + 1 < p_end) load_x(p + 1, mb ^ 1);
-
-    // ---- softmax of query `row` over its 128 in-window keys
-    const int qs = c0 * kAttnM + row;  // query slot
-    const bool qvalid = qs < a.n;
-    const float* ki = kinv + mb * kAttnKeys;
-    const int32_t* kp = kpos + mb * kAttnKeys;
-    const int qpos = kp[row + kAttnM];
-    float l[128];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      uint32_t v[32];
-      tmem_ld32(tm_s + tl + wcol + b * 32, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const int j = wcol + b * 32 + k;  // key column in the window
-        const int ks = k0 + j;            // key slot
-        float x = __uint_as_float(v[k]) * ki[j] * qk_scale;
-        if (j == row + kAttnM) x = kSelfLogit;
-        const bool keep = ks >= 0 && ks < a.n && !(a.causal && kp[j] > qpos);
-        x = keep ? x : -INFINITY;
-        l[b * 32 + k] = x;
-        mx = fmaxf(mx, x);
-      }
-    }
-    // the query's own slot is always in its window, so mx is finite
-    float sum = 0.f;
-    const float mx2 = mx * kLog2e;
-#pragma unroll
-    for (int k = 0; k < 128; ++k) {
-      const float e = exp2f(fmaf(l[k], kLog2e, -mx2));  // 0 for removed keys (-inf)
-      l[k] = e;
-      sum += e;
-    }
-    if (warp < 2)
-      store_p_row<0>(l, tm_s + tl);
-    else
-      store_p_row<kAttnM>(l, tm_s + tl);
-    tmem_wait_st();
-    tc_fence_before();
-    if (!__syncthreads_and(ok)) break;
-
-    // ---- MMA 2: O = P V
-    if (tid == 0) {
-      tc_fence_after();
-      if (mbar_wait(v_full, ph)) {
-        const uint32_t va = smem_u32(vt);
+        mma_commit(sfull + s);
+        mma_commit(xfree + s);
+        return true;
+      };
+      auto issue_pv = [&](int i) {
+        const int s = i & 1, k = i >> 1;
+        if (!mbar_wait(pready + s, k & 1)) return false;
+        if (!mbar_wait(vfull + s, k & 1)) return false;
+        if (i > 0 && !mbar_wait(ofree, (i - 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t va = smem_u32(vt + s * TILE);
 #pragma unroll
         for (int kk = 0; kk < kAttnKeys / 16; ++kk) {
           const uint64_t bd = desc_mnmajor_sw128(va + kk * 16 * 128, BOX);
-          mma_bf16_ts(tm_o, tm_s + kk * 8, bd, idesc_o, kk > 0 ? 1u : 0u);
+          mma_bf16_ts(tm_o, tmem + s * 192 + kk * 8, bd, idesc_o, kk > 0 ? 1u : 0u);
         }
-        mma_commit(o_done);
-      } else {
-        ok = false;
+        mma_commit(ofull);
+        mma_commit(vfree + s);
+        mma_commit(sfree + s);
+        return true;
+      };
+      bool ok = issue_s(0);
+      for (int i = 0; ok && i < nu && !*abort_flag; ++i)
+        ok = (i + 1 >= nu || issue_s(i + 1)) && issue_pv(i);
+      if (!ok) fail();
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ softmax
+    const int q = warp & 3;       // TMEM lane quadrant
+    const int st = tid - 64;      // 0..127 among the softmax threads
+    const int row = q * 32 + lane;
+    const int wcol = q < 2 ? 0 : kAttnM;  // first in-window key column
+    const uint32_t tl = (uint32_t)(q * 32) << 16;
+    const float c_scale = kLog2e / sqrtf((float)D);
+    for (int i = 0; i < nu; ++i) {
+      const int s = i & 1, k = i >> 1;
+      if (!mbar_wait(sfull + s, k & 1)) { fail(); break; }
+      tc_fence_after();
+      const int64_t seg = unit_seg(i);
+      const int c0 = unit_c0(i);
+      const int k0 = (c0 - 1) * kAttnM;
+      // per-key table: logit scale (log2 units) and position; keys outside
+      // [0, n) get a position that every query's test rejects
+      float2* kt = ktab + s * kAttnKeys;
+      for (int j = st; j < kAttnKeys; j += 128) {
+        const int ks = k0 + j;
+        const bool valid = ks >= 0 && ks < a.n;
+        kt[j] = make_float2(valid ? kinv[s * kAttnKeys + j] * c_scale : 0.f,
+                            __int_as_float(valid ? kpos[s * kAttnKeys + j] : kNoKey));
+      }
+      const float qinv = kinv[s * kAttnKeys + kAttnM + row];
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
+      if (lane == 0) mbar_arrive(xfree + s);  // metadata of this stage consumed
+      const int qpos = __float_as_int(kt[kAttnM + row].y);
+      // stabiliser: ||q|| log2(e) / sqrt(d) bounds every logit of the row
+      float bound = qinv > 0.f ? c_scale / qinv : 0.f;
+      const uint32_t ts = tmem + tl + s * 192;
+      auto visible = [&](int pj) {
+        if (CAUSAL) return pj < qpos;            // earlier positions only (not self)
+        return pj != qpos && pj != kNoKey;       // every valid key but self
+      };
+      if (__any_sync(0xffffffffu, bound > kAttnBoundMax)) {
+        // rare: exact row maximum as the stabiliser for those rows
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int b = 0; b < 4; ++b) {
+          uint32_t v[32];
+          tmem_ld32(ts + wcol + b * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float2 t = kt[wcol + b * 32 + c];
+            if (visible(__float_as_int(t.y))) mx = fmaxf(mx, __uint_as_float(v[c]) * t.x);
+          }
+        }
+        if (bound > kAttnBoundMax) bound = mx == -INFINITY ? 0.f : mx;
+      }
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll 1
+      for (int b = 0; b < 4; ++b) {
+        uint32_t v[32];
+        tmem_ld32(ts + wcol + b * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float2 t0 = kt[wcol + b * 32 + c];
+          const float2 t1 = kt[wcol + b * 32 + c + 1];
+          const float l0 = fmaf(__uint_as_float(v[c]), t0.x, -bound);
+          const float l1 = fmaf(__uint_as_float(v[c + 1]), t1.x, -bound);
+          const float e0 = visible(__float_as_int(t0.y)) ? exp2f(l0) : 0.f;
+          const float e1 = visible(__float_as_int(t1.y)) ? exp2f(l1) : 0.f;
+          sum0 += e0;
+          sum1 += e1;
+          pk[c >> 1] = pack_bf16x2(e0, e1);
+        }
+        // P column c holds keys 2c, 2c+1: chunk b lands in columns
+        // [wcol/2 + 16b, wcol/2 + 16b + 16), behind every S column still unread
+        tmem_st16(ts + wcol / 2 + b * 16, pk);
+      }
+      uint32_t z[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) z[c] = 0u;
+      tmem_st16(ts + (q < 2 ? 64 : 0), z);  // P outside this row's window
+      tmem_st16(ts + (q < 2 ? 80 : 16), z);
+      tmem_wait_st();
+      const float sum = sum0 + sum1;
+      const int qs = c0 * kAttnM + row;
+      // lse over the visible keys and the self logit; exp(-1e5) vanishes
+      // unless the row sees nothing else
+      if (qs < a.n)
+        a.lse_s[seg * a.n + qs] = sum > 0.f ? (bound + log2f(sum)) * 0.6931471805599453f
+                                            : kSelfLogit;
+      rstat[(i % kAttnStats) * 128 + row] = sum > 0.f ? 1.0f / sum : -1.f;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(pready + s);
+        mbar_arrive(statf + (i % kAttnStats));
       }
     }
-    if (!__syncthreads_and(ok)) break;
-    if (!mbar_wait(o_done, ph)) ok = false;
-    tc_fence_after();
-    if (tid == 0 && ok && p + 1 < p_end) load_v(p + 1);  // v tile is free again
-
-    // ---- O / sum and lse
-    if (qvalid) {
-      const float inv = 1.0f / sum;
-      float* orow = a.out_s + (seg * a.n + qs) * (int64_t)D;
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t tl = (uint32_t)(q * 32) << 16;
+    for (int i = 0; i < nu; ++i) {
+      if (!mbar_wait(ofull, i & 1) || !mbar_wait(statf + (i % kAttnStats), (i / kAttnStats) & 1)) {
+        fail();
+        break;
+      }
+      tc_fence_after();
+      uint32_t o[D / 32][32];
 #pragma unroll
-      for (int b = 0; b < D / 32; ++b) {
-        uint32_t v[32];
-        tmem_ld32(tm_o + tl + b * 32, v);
-        tmem_wait_ld();
+      for (int b = 0; b < D / 32; ++b) tmem_ld32(tm_o + tl + b * 32, o[b]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ofree);
+      const int64_t seg = unit_seg(i);
+      const int qs = unit_c0(i) * kAttnM + row;
+      if (qs < a.n) {
+        const float inv = rstat[(i % kAttnStats) * 128 + row];
+        float* orow = a.out_s + (seg * a.n + qs) * (int64_t)D;
+        if (inv > 0.f) {
 #pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-          float4 o;
-          o.x = __uint_as_float(v[k]) * inv;
-          o.y = __uint_as_float(v[k + 1]) * inv;
-          o.z = __uint_as_float(v[k + 2]) * inv;
-          o.w = __uint_as_float(v[k + 3]) * inv;
-          *reinterpret_cast<float4*>(orow + b * 32 + k) = o;
+          for (int c = 0; c < D; c += 4)
+            *reinterpret_cast<float4*>(orow + c) = make_float4(
+                __uint_as_float(o[c / 32][c % 32]) * inv,
+                __uint_as_float(o[c / 32][c % 32 + 1]) * inv,
+                __uint_as_float(o[c / 32][c % 32 + 2]) * inv,
+                __uint_as_float(o[c / 32][c % 32 + 3]) * inv);
+        } else {  // only the token itself is visible: its own value row
+          const uint4* vr = reinterpret_cast<const uint4*>(a.vs + (seg * a.n + qs) * (int64_t)D);
+          for (int c = 0; c < D / 8; ++c) {
+            float f[8];
+            Vec16<__nv_bfloat16>::unpack(vr[c], f);
+            *reinterpret_cast<float4*>(orow + 8 * c) = make_float4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<float4*>(orow + 8 * c + 4) = make_float4(f[4], f[5], f[6], f[7]);
+          }
         }
       }
-      a.lse_s[seg * a.n + qs] = mx + logf(sum);
-    } else {
-      // keep the warp's tcgen05.ld calls uniform
-#pragma unroll
-      for (int b = 0; b < D / 32; ++b) {
-        uint32_t v[32];
-        tmem_ld32(tm_o + tl + b * 32, v);
-        tmem_wait_ld();
-      }
     }
-    tc_fence_before();
-    if (!__syncthreads_and(ok)) break;
   }
-  if (!ok && tid == 0) record_status(a.hdr, 5u /* LSH_ERR_TIMEOUT */);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kAttnTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
 inline size_t attn_tc_smem(int D) {
   const size_t tile = (size_t)(D / 64) * kAttnKeys * 128;
-  size_t s = 1024 + 2 * tile + 2 * kAttnKeys * 4 * 2 + 64;
-  // at most two CTAs per SM: each holds 256 of the 512 TMEM columns
-  return s < 80 * 1024 ? 80 * 1024 : s;
+  return 1024 + 4 * tile + 2 * kAttnKeys * (4 + 4 + 8) + kAttnStats * 128 * 4 + 256;
 }
 
 }  // namespace lsh

@@ -73,74 +73,73 @@ inline HashTcPlan hash_tc_plan(int d, int nb, int rounds) {
 // R [rounds][d][half] -> Rt [rounds][ch * nc][d]: K-major rows for the MMA's
 // B operand, each round padded with zero rows to whole chunks of nc. Also,
 // per round, an upper bound of max_j ||R_j|| (float bits in rnorm_bits[r],
-// zeroed before the launch).
-// grid (ceil(ch * nc / 128), rounds), block 128.
-__global__ void __launch_bounds__(128)
+// zeroed before the launch). A CTA transposes 32 columns through shared
+// memory. grid (ceil(ch * nc / 32), rounds), block 256.
+__global__ void __launch_bounds__(256)
     k_hash_prep(const __nv_bfloat16* __restrict__ R, __nv_bfloat16* __restrict__ Rt,
                 uint32_t* __restrict__ rnorm_bits, int d, int half, int rows_per_round) {
+  __shared__ __nv_bfloat16 tile[128][34];  // [k][column], padded rows
   const int r = blockIdx.y;
-  const int j = blockIdx.x * 128 + threadIdx.x;
-  if (j >= rows_per_round) return;
-  __nv_bfloat16* dst = Rt + ((int64_t)r * rows_per_round + j) * d;
-  if (j >= half) {
-    for (int k = 0; k < d; ++k) dst[k] = __float2bfloat16_rn(0.f);
-    return;
+  const int j0 = blockIdx.x * 32;
+  const __nv_bfloat16* src = R + (int64_t)r * d * half;
+  for (int e = threadIdx.x; e < d * 32; e += blockDim.x) {
+    const int k = e >> 5, jj = e & 31;
+    tile[k][jj] = (j0 + jj < half) ? src[(int64_t)k * half + j0 + jj] : __float2bfloat16_rn(0.f);
   }
-  const __nv_bfloat16* src = R + (int64_t)r * d * half + j;
-  double ss = 0.0;
-  for (int k = 0; k < d; ++k) {
-    const __nv_bfloat16 e = src[(int64_t)k * half];
-    dst[k] = e;
-    const double f = (double)__bfloat162float(e);
-    ss += f * f;
+  __syncthreads();
+  if (threadIdx.x < 32 && j0 + threadIdx.x < half) {
+    double ss = 0.0;
+    for (int k = 0; k < d; ++k) {
+      const double f = (double)__bfloat162float(tile[k][threadIdx.x]);
+      ss += f * f;
+    }
+    const float nrm = __double2float_ru(sqrt(ss));  // rounded up: an upper bound
+    atomicMax(rnorm_bits + r, __float_as_uint(nrm));  // non-negative floats order as uints
   }
-  const float nrm = __double2float_ru(sqrt(ss));  // rounded up: an upper bound
-  atomicMax(rnorm_bits + r, __float_as_uint(nrm));  // non-negative floats order as uints
+  __nv_bfloat16* dst = Rt + ((int64_t)r * rows_per_round + j0) * d;
+  for (int e = threadIdx.x; e < d * 32; e += blockDim.x) {
+    const int jj = e / d, k = e % d;
+    if (j0 + jj < rows_per_round) dst[(int64_t)jj * d + k] = tile[k][jj];
+  }
 }
 
 // ---------------------------------------------------------------------------
-// Exact fp64 re-decision of queued (token, round) pairs; one warp per entry.
-// entries: (bh * n + t) << 5 | r. Count in hdr->hash_refined.
-__global__ void __launch_bounds__(256)
-    k_hash_refine(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ R,
+// Exact fp64 re-decision of queued (token, round) pairs; one CTA per entry.
+// entries: (bh * n + t) << 5 | r; count in hdr->hash_refined. Each thread
+// sums whole columns of the transposed rotation in increasing k, so every
+// p_j is the same fp64 number a sequential evaluation of the definition gives
+// (bf16 products are exact in fp64).
+template <int D>
+__global__ void __launch_bounds__(128)
+    k_hash_refine(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Rt,
                   const uint64_t* __restrict__ entries, int32_t* __restrict__ buckets, int n,
-                  int d, int nb, int rounds, const WsHeader* __restrict__ hdr) {
+                  int nb, int rounds, int rows_per_round, const WsHeader* __restrict__ hdr) {
+  __shared__ double xs[D];
+  __shared__ double wv[4];
+  __shared__ int wi[4];
   const int half = nb / 2;
   const uint32_t count = hdr->hash_refined;
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t e = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); e < count;
-       e += warps) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (uint32_t e = blockIdx.x; e < count; e += gridDim.x) {
     const uint64_t code = entries[e];
     const int r = (int)(code & 31);
     const int64_t row = (int64_t)(code >> 5);  // bh * n + t
-    const int64_t bh = row / n;
-    const int t = (int)(row % n);
-    const __nv_bfloat16* xr = x + row * d;
-    const __nv_bfloat16* Rr = R + (int64_t)r * d * half;
+    if (tid < D) xs[tid] = (double)__bfloat162float(x[row * D + tid]);
+    __syncthreads();
     double bv = -INFINITY;
     int bi = 0x7fffffff;
-    for (int j0 = 0; j0 < half; j0 += 32 * 8) {
-      double acc[8];
+    for (int j = tid; j < half; j += 128) {
+      const uint4* rr = reinterpret_cast<const uint4*>(Rt + ((int64_t)r * rows_per_round + j) * D);
+      double acc = 0.0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-      for (int k = 0; k < d; ++k) {
-        const double xk = (double)__bfloat162float(xr[k]);
-        const __nv_bfloat16* Rk = Rr + (int64_t)k * half;
+      for (int c = 0; c < D / 8; ++c) {
+        float f[8];
+        Vec16<__nv_bfloat16>::unpack(__ldg(rr + c), f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int j = j0 + i * 32 + lane;
-          if (j < half) acc[i] = fma(xk, (double)__bfloat162float(Rk[j]), acc[i]);
-        }
+        for (int u = 0; u < 8; ++u) acc = fma(xs[c * 8 + u], (double)f[u], acc);
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int j = j0 + i * 32 + lane;
-        if (j < half) {
-          argmax_update(acc[i], j, bv, bi);
-          argmax_update(-acc[i], half + j, bv, bi);
-        }
-      }
+      argmax_update(acc, j, bv, bi);
+      argmax_update(-acc, half + j, bv, bi);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -148,7 +147,18 @@ __global__ void __launch_bounds__(256)
       const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
       argmax_update(ov, oi, bv, bi);
     }
-    if (lane == 0) buckets[(bh * rounds + r) * n + t] = bi;
+    if (lane == 0) {
+      wv[warp] = bv;
+      wi[warp] = bi;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      for (int w = 1; w < 4; ++w) argmax_update(wv[w], wi[w], bv, bi);
+      const int64_t bh = row / n;
+      const int t = (int)(row % n);
+      buckets[(bh * rounds + r) * n + t] = bi;
+    }
+    __syncthreads();
   }
 }
 
@@ -178,7 +188,21 @@ struct Top2 {
     sv = gt ? v : sv;
     m1 = gt ? a : m1;
   }
+  // Fold another tracker in: the larger first value wins (lower index on a
+  // tie); the second value is the largest of the rest.
+  __device__ __forceinline__ void merge(float om1, float om2, int oidx, float osv) {
+    if (om1 > m1 || (om1 == m1 && oidx < idx)) {
+      m2 = fmaxf(fmaxf(om2, m2), m1);
+      m1 = om1;
+      idx = oidx;
+      sv = osv;
+    } else {
+      m2 = fmaxf(fmaxf(om2, m2), om1);
+    }
+  }
 };
+
+constexpr int kHashLanesIlp = 4;  // independent trackers per thread (ILP)
 
 template <int D>
 __global__ void __launch_bounds__(kHashWarps * 32, 1)
@@ -333,8 +357,9 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
       }
       bool stop = false;
       for (int rl = 0; rl < gr; ++rl, ++rc) {
-        Top2 st;
-        st.reset();
+        Top2 st[kHashLanesIlp];
+#pragma unroll
+        for (int i = 0; i < kHashLanesIlp; ++i) st[i].reset();
         for (int c = 0; ok && c < p.ch; ++c, ++u) {
           const int ab = u & 1, uk = u >> 1;
           if (!mbar_wait(acc_full + ab, uk & 1)) {
@@ -344,43 +369,49 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
           }
           tc_fence_after();
           const uint32_t tbase = tmem + tlane + ab * p.tmem_cols;
-          for (int b = h; b < nbatch; b += 2) {
-            uint32_t v[16];
-            tmem_ld16(tbase + b * 16, v);
+          // this warp's 16-column batches are h, h + 2, ...: four loads in
+          // flight per wait
+          for (int i0 = 0; 2 * i0 + h < nbatch; i0 += 4) {
+            uint32_t v[4][16];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (h + 2 * (i0 + i) < nbatch) tmem_ld16(tbase + (h + 2 * (i0 + i)) * 16, v[i]);
             tmem_wait_ld();
-            const int j0 = c * p.nc + b * 16;
-            if (j0 + 16 <= p.half) {
 #pragma unroll
-              for (int k = 0; k < 16; ++k) st.add(__uint_as_float(v[k]), j0 + k);
-            } else {
+            for (int i = 0; i < 4; ++i) {
+              const int b = h + 2 * (i0 + i);
+              if (b < nbatch) {
+                const int j0 = c * p.nc + b * 16;
+                if (j0 + 16 <= p.half) {
 #pragma unroll
-              for (int k = 0; k < 16; ++k)
-                if (j0 + k < p.half) st.add(__uint_as_float(v[k]), j0 + k);
+                  for (int k = 0; k < 16; ++k)
+                    st[k % kHashLanesIlp].add(__uint_as_float(v[i][k]), j0 + k);
+                } else {
+#pragma unroll
+                  for (int k = 0; k < 16; ++k)
+                    if (j0 + k < p.half)
+                      st[k % kHashLanesIlp].add(__uint_as_float(v[i][k]), j0 + k);
+                }
+              }
             }
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty + ab);
+          if (lane == 0) mbar_arrive(acc_empty + ab);  // accumulator free for the next MMA
         }
+#pragma unroll
+        for (int i = 1; i < kHashLanesIlp; ++i) st[0].merge(st[i].m1, st[i].m2, st[i].idx, st[i].sv);
         // combine the two warps of this quadrant, then decide
         float4* slot = comb + ((rc & 1) * 4 + q) * 32 + lane;
-        if (h == 1) *slot = make_float4(st.m1, st.m2, __int_as_float(st.idx), st.sv);
+        if (h == 1) *slot = make_float4(st[0].m1, st[0].m2, __int_as_float(st[0].idx), st[0].sv);
         asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
         stop = *abort_flag != 0;
         if (stop) break;
         if (h == 0) {
           const float4 o = *slot;
-          const int oidx = __float_as_int(o.z);
-          float m1 = st.m1, m2, sv = st.sv;
-          int idx = st.idx;
-          if (o.x > st.m1 || (o.x == st.m1 && oidx < st.idx)) {
-            m2 = fmaxf(fmaxf(o.y, st.m2), st.m1);
-            m1 = o.x;
-            idx = oidx;
-            sv = o.w;
-          } else {
-            m2 = fmaxf(fmaxf(o.y, st.m2), o.x);
-          }
+          st[0].merge(o.x, o.y, __float_as_int(o.z), o.w);
+          const float m1 = st[0].m1, m2 = st[0].m2, sv = st[0].sv;
+          const int idx = st[0].idx;
           if (t < a.n) {
             const int r = r0 + rl;
             const float tau = kTieFactor * (float)D * 1.1920929e-7f * xnorm * rnorm[r];

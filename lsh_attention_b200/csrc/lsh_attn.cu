@@ -149,8 +149,8 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
   __nv_bfloat16* rt = at<__nv_bfloat16>(ws, L.rt);
   uint64_t* refine = at<uint64_t>(ws, L.refine);
   const int rows_per_round = p.ch * p.nc;
-  dim3 pg((rows_per_round + 127) / 128, D.rounds);
-  k_hash_prep<<<pg, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(R), rt, hdr->pad, D.d, p.half,
+  dim3 pg((rows_per_round + 31) / 32, D.rounds);
+  k_hash_prep<<<pg, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(R), rt, hdr->pad, D.d, p.half,
                                   rows_per_round);
   CUtensorMap tmx, tmr;
   if (!make_tmap_bf16_2d(&tmx, x, D.d, (uint64_t)D.BH * D.n, (uint64_t)D.d * 2, 64, kHashTile) ||
@@ -185,9 +185,12 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
       return LSH_ERR_CUDA;
     kern<<<grid, kHashWarps * 32, p.smem, st>>>(tmx, tmr, a, p);
   }
-  k_hash_refine<<<2 * sms, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
-                                         static_cast<const __nv_bfloat16*>(R), refine, buckets,
-                                         D.n, D.d, D.nb, D.rounds, hdr);
+  if (D.d == 64)
+    k_hash_refine<64><<<8 * sms, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine,
+                                               buckets, D.n, D.nb, D.rounds, rows_per_round, hdr);
+  else
+    k_hash_refine<128><<<8 * sms, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine,
+                                                buckets, D.n, D.nb, D.rounds, rows_per_round, hdr);
   return last_cuda();
 }
 
@@ -248,6 +251,17 @@ inline bool attn_tc_supported(const Dims& D) {
          D.S * (int64_t)D.n < (int64_t(1) << 31);
 }
 
+template <int DD, bool CAUSAL>
+lsh_status launch_attn_tc_k(const CUtensorMap& tmx, const CUtensorMap& tmv, const AttnTcArgs& a,
+                            unsigned grid, size_t smem, cudaStream_t st) {
+  auto kern = k_attn_tc<DD, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LSH_ERR_CUDA;
+  kern<<<grid, kAttnWarps * 32, smem, st>>>(tmx, tmv, a);
+  return last_cuda();
+}
+
 lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
                           const float* invnorm, float* out_s, float* lse_s, WsHeader* hdr,
                           cudaStream_t st) {
@@ -259,6 +273,7 @@ lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const i
   AttnTcArgs a;
   a.invnorm = invnorm;
   a.perm = perm;
+  a.vs = static_cast<const __nv_bfloat16*>(vs);
   a.out_s = out_s;
   a.lse_s = lse_s;
   a.hdr = hdr;
@@ -266,24 +281,15 @@ lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const i
   a.causal = D.causal;
   a.pairs_per_seg = (D.n / kAttnM + 1) / 2;
   a.pairs = D.S * a.pairs_per_seg;
-  const int64_t ctas_max = 2 * (int64_t)sm_count();
+  const int64_t ctas_max = (int64_t)sm_count();
   a.pairs_per_cta = (a.pairs + ctas_max - 1) / ctas_max;
   const unsigned grid = (unsigned)((a.pairs + a.pairs_per_cta - 1) / a.pairs_per_cta);
   const size_t smem = attn_tc_smem(D.d);
-  if (D.d == 64) {
-    auto kern = k_attn_tc<64>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return LSH_ERR_CUDA;
-    kern<<<grid, 128, smem, st>>>(tmx, tmv, a);
-  } else {
-    auto kern = k_attn_tc<128>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return LSH_ERR_CUDA;
-    kern<<<grid, 128, smem, st>>>(tmx, tmv, a);
-  }
-  return last_cuda();
+  if (D.d == 64)
+    return D.causal ? launch_attn_tc_k<64, true>(tmx, tmv, a, grid, smem, st)
+                    : launch_attn_tc_k<64, false>(tmx, tmv, a, grid, smem, st);
+  return D.causal ? launch_attn_tc_k<128, true>(tmx, tmv, a, grid, smem, st)
+                  : launch_attn_tc_k<128, false>(tmx, tmv, a, grid, smem, st);
 }
 
 template <typename T, int DD>

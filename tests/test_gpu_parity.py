@@ -216,6 +216,8 @@ EDGE = [
     ("chunk-128", 1, 2, 1024, 128, 32, 128, 2, True, "bf16"),
     ("many-rounds", 1, 1, 256, 64, 8, 32, 16, True, "f32"),
     ("max-buckets", 1, 1, 8192, 64, 4096, 64, 1, True, "bf16"),
+    ("noncausal-bf16-d128", 1, 2, 1024, 128, 32, 64, 2, False, "bf16"),
+    ("noncausal-bf16-d64", 2, 1, 640, 64, 16, 64, 3, False, "bf16"),
 ]
 
 
@@ -237,6 +239,27 @@ def test_edge_cases(case):
                                    buckets=bk.cuda())
     check_close(out.float().cpu().numpy(), ref_out, dt, f"{name} out")
     check_close(lse.cpu().numpy(), ref_lse, dt, f"{name} lse")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_reversed_buckets_self_only_rows(causal):
+    """Bucket ids that reverse the order: slot s holds position n-1-s, so in
+    causal mode the last slot of every chunk sees nothing but itself."""
+    n = 2048
+    w = I.Workload("reversed", 1, 2, n, 128, n, 64, 1, causal, "bf16")
+    x, v = I.make_qkv(w)
+    bk = torch.arange(n - 1, -1, -1, dtype=torch.int32).repeat(1, 2, 1, 1)
+    ref_out, ref_lse, _ = oracle.forward(x, v, I.make_rotations(w), 64, causal, buckets=bk)
+    if causal:
+        assert (ref_lse == -1e5).sum() >= 2 * n // 64
+    xg, vg = to_gpu(x, v)
+    out, lse = lb.lsh_attn_forward(xg, vg, None, n_buckets=n, chunk=64, causal=causal,
+                                   buckets=bk.cuda())
+    check_close(out.float().cpu().numpy(), ref_out, "bf16", "reversed out")
+    check_close(lse.cpu().numpy(), ref_lse, "bf16", "reversed lse")
+    if causal:
+        self_only = ref_lse == -1e5
+        np.testing.assert_array_equal(lse.cpu().numpy()[self_only], -1e5)
 
 
 def test_all_tokens_one_bucket():
