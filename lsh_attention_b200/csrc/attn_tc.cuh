@@ -23,7 +23,9 @@
 //               dead S columns) as soon as it is computed; the row sum goes to
 //               the epilogue. A row whose only visible key is itself (the -1e5
 //               self logit) is flagged: its output is v of the query itself.
-//   warps 6..9  epilogue: O from TMEM, divided by the row sum, stored fp32
+//   warps 6..9  epilogue: O from TMEM, divided by the row sum, staged per warp
+//               in a 4 KB swizzled buffer (32 rows x 32 fp32) and written by
+//               TMA bulk stores, so every 128-byte line leaves the SM whole
 // TMEM: S[0] = [0, 192), S[1] = [192, 384), O = [384, 384 + d).
 #pragma once
 
@@ -60,7 +62,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmv,
-              AttnTcArgs a) {
+              const __grid_constant__ CUtensorMap tmo, AttnTcArgs a) {
   using namespace sm100;
   constexpr int KH = D / 64;
   constexpr uint32_t BOX = kAttnKeys * 128;
@@ -72,7 +74,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* xt = base;                                          // [2][KH][192][128 B]
   unsigned char* vt = base + 2 * TILE;                               // [2][KH][192][128 B]
-  float* kinv = reinterpret_cast<float*>(base + 4 * TILE);           // [2][192]
+  unsigned char* ostage = base + 4 * TILE;                           // [4 warps][32][128 B]
+  float* kinv = reinterpret_cast<float*>(ostage + 4 * 32 * 128);     // [2][192]
   int32_t* kpos = reinterpret_cast<int32_t*>(kinv + 2 * kAttnKeys);  // [2][192]
   float2* ktab = reinterpret_cast<float2*>(kpos + 2 * kAttnKeys);    // [2][192] (scale, pos)
   float* rstat = reinterpret_cast<float*>(ktab + 2 * kAttnKeys);     // [4][128]
@@ -312,29 +315,44 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(ofree);
       const int64_t seg = unit_seg(i);
-      const int qs = unit_c0(i) * kAttnM + row;
-      if (qs < a.n) {
+      const int qs0 = unit_c0(i) * kAttnM + q * 32;  // first query slot of this warp
+      if (qs0 < a.n) {  // n % 64 == 0: a warp's 32 rows are all valid or all not
         const float inv = rstat[(i % kAttnStats) * 128 + row];
-        float* orow = a.out_s + (seg * a.n + qs) * (int64_t)D;
-        if (inv > 0.f) {
+        const uint4* vr = reinterpret_cast<const uint4*>(a.vs + (seg * a.n + qs0 + lane) * (int64_t)D);
+        unsigned char* stg = ostage + (warp - 6) * 32 * 128;
 #pragma unroll
-          for (int c = 0; c < D; c += 4)
-            *reinterpret_cast<float4*>(orow + c) = make_float4(
-                __uint_as_float(o[c / 32][c % 32]) * inv,
-                __uint_as_float(o[c / 32][c % 32 + 1]) * inv,
-                __uint_as_float(o[c / 32][c % 32 + 2]) * inv,
-                __uint_as_float(o[c / 32][c % 32 + 3]) * inv);
-        } else {  // only the token itself is visible: its own value row
-          const uint4* vr = reinterpret_cast<const uint4*>(a.vs + (seg * a.n + qs) * (int64_t)D);
-          for (int c = 0; c < D / 8; ++c) {
-            float f[8];
-            Vec16<__nv_bfloat16>::unpack(vr[c], f);
-            *reinterpret_cast<float4*>(orow + 8 * c) = make_float4(f[0], f[1], f[2], f[3]);
-            *reinterpret_cast<float4*>(orow + 8 * c + 4) = make_float4(f[4], f[5], f[6], f[7]);
+        for (int b = 0; b < D / 32; ++b) {
+          if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
+          __syncwarp();
+          // row `lane`, 16-byte chunk c goes to slot c ^ (lane % 8) (128-byte swizzle)
+          unsigned char* line = stg + lane * 128;
+          if (inv > 0.f) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<float4*>(line + ((c ^ (lane & 7)) << 4)) = make_float4(
+                  __uint_as_float(o[b][4 * c]) * inv, __uint_as_float(o[b][4 * c + 1]) * inv,
+                  __uint_as_float(o[b][4 * c + 2]) * inv, __uint_as_float(o[b][4 * c + 3]) * inv);
+          } else {  // only the token itself is visible: its own value row
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float f[8];
+              Vec16<__nv_bfloat16>::unpack(vr[b * 4 + c], f);
+              *reinterpret_cast<float4*>(line + (((2 * c) ^ (lane & 7)) << 4)) =
+                  make_float4(f[0], f[1], f[2], f[3]);
+              *reinterpret_cast<float4*>(line + (((2 * c + 1) ^ (lane & 7)) << 4)) =
+                  make_float4(f[4], f[5], f[6], f[7]);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmo, stg, b * 32, (int)(seg * a.n) + qs0);
+            bulk_commit();
           }
         }
       }
     }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -346,7 +364,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
 
 inline size_t attn_tc_smem(int D) {
   const size_t tile = (size_t)(D / 64) * kAttnKeys * 128;
-  return 1024 + 4 * tile + 2 * kAttnKeys * (4 + 4 + 8) + kAttnStats * 128 * 4 + 256;
+  return 1024 + 4 * tile + 4 * 32 * 128 + 2 * kAttnKeys * (4 + 4 + 8) + kAttnStats * 128 * 4 +
+         256;
 }
 
 }  // namespace lsh

@@ -252,23 +252,25 @@ inline bool attn_tc_supported(const Dims& D) {
 }
 
 template <int DD, bool CAUSAL>
-lsh_status launch_attn_tc_k(const CUtensorMap& tmx, const CUtensorMap& tmv, const AttnTcArgs& a,
-                            unsigned grid, size_t smem, cudaStream_t st) {
+lsh_status launch_attn_tc_k(const CUtensorMap& tmx, const CUtensorMap& tmv,
+                            const CUtensorMap& tmo, const AttnTcArgs& a, unsigned grid,
+                            size_t smem, cudaStream_t st) {
   auto kern = k_attn_tc<DD, CAUSAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return LSH_ERR_CUDA;
-  kern<<<grid, kAttnWarps * 32, smem, st>>>(tmx, tmv, a);
+  kern<<<grid, kAttnWarps * 32, smem, st>>>(tmx, tmv, tmo, a);
   return last_cuda();
 }
 
 lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
                           const float* invnorm, float* out_s, float* lse_s, WsHeader* hdr,
                           cudaStream_t st) {
-  CUtensorMap tmx, tmv;
+  CUtensorMap tmx, tmv, tmo;
   const uint64_t rows = (uint64_t)D.S * D.n;
   if (!make_tmap_bf16_2d(&tmx, xs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys) ||
-      !make_tmap_bf16_2d(&tmv, vs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys))
+      !make_tmap_bf16_2d(&tmv, vs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys) ||
+      !make_tmap_f32_2d(&tmo, out_s, D.d, rows, (uint64_t)D.d * 4, 32, 32))
     return LSH_ERR_CUDA;
   AttnTcArgs a;
   a.invnorm = invnorm;
@@ -286,10 +288,10 @@ lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const i
   const unsigned grid = (unsigned)((a.pairs + a.pairs_per_cta - 1) / a.pairs_per_cta);
   const size_t smem = attn_tc_smem(D.d);
   if (D.d == 64)
-    return D.causal ? launch_attn_tc_k<64, true>(tmx, tmv, a, grid, smem, st)
-                    : launch_attn_tc_k<64, false>(tmx, tmv, a, grid, smem, st);
-  return D.causal ? launch_attn_tc_k<128, true>(tmx, tmv, a, grid, smem, st)
-                  : launch_attn_tc_k<128, false>(tmx, tmv, a, grid, smem, st);
+    return D.causal ? launch_attn_tc_k<64, true>(tmx, tmv, tmo, a, grid, smem, st)
+                    : launch_attn_tc_k<64, false>(tmx, tmv, tmo, a, grid, smem, st);
+  return D.causal ? launch_attn_tc_k<128, true>(tmx, tmv, tmo, a, grid, smem, st)
+                  : launch_attn_tc_k<128, false>(tmx, tmv, tmo, a, grid, smem, st);
 }
 
 template <typename T, int DD>
