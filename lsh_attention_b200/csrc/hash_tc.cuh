@@ -104,59 +104,88 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
-// Exact fp64 re-decision of queued (token, round) pairs; one CTA per entry.
-// entries: (bh * n + t) << 5 | r; count in hdr->hash_refined. Each thread
-// sums whole columns of the transposed rotation in increasing k, so every
-// p_j is the same fp64 number a sequential evaluation of the definition gives
-// (bf16 products are exact in fp64).
+// Exact fp64 re-decision of queued tokens. The queue of round r holds row
+// indices bh * n + t at queue + r * cap; its length is count[r]. A CTA takes
+// kRefineBatch entries of one round at a time, so each element of the
+// transposed rotation is converted to fp64 once per batch. Every thread sums
+// whole columns in increasing k, so p_j is the same fp64 number a sequential
+// evaluation of the definition gives (bf16 products are exact in fp64).
+// grid (ctas per round, rounds), block 128.
+constexpr int kRefineBatch = 8;
+
 template <int D>
 __global__ void __launch_bounds__(128)
     k_hash_refine(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Rt,
-                  const uint64_t* __restrict__ entries, int32_t* __restrict__ buckets, int n,
-                  int nb, int rounds, int rows_per_round, const WsHeader* __restrict__ hdr) {
-  __shared__ double xs[D];
-  __shared__ double wv[4];
-  __shared__ int wi[4];
+                  const uint64_t* __restrict__ queue, int64_t cap, int32_t* __restrict__ buckets,
+                  int n, int nb, int rounds, int rows_per_round, const WsHeader* __restrict__ hdr) {
+  constexpr int E = kRefineBatch;
+  __shared__ double xs[E][D];
+  __shared__ double wv[4][E];
+  __shared__ int wi[4][E];
+  const int r = blockIdx.y;
   const int half = nb / 2;
-  const uint32_t count = hdr->hash_refined;
+  const uint32_t count = hdr->pad[16 + r];
+  const uint64_t* qr = queue + r * cap;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (uint32_t e = blockIdx.x; e < count; e += gridDim.x) {
-    const uint64_t code = entries[e];
-    const int r = (int)(code & 31);
-    const int64_t row = (int64_t)(code >> 5);  // bh * n + t
-    if (tid < D) xs[tid] = (double)__bfloat162float(x[row * D + tid]);
+  const __nv_bfloat16* Rr = Rt + (int64_t)r * rows_per_round * D;
+  for (uint32_t e0 = blockIdx.x * E; e0 < count; e0 += gridDim.x * E) {
+    const int ne = min(E, (int)(count - e0));
+    for (int i = tid; i < E * D; i += 128) {
+      const int e = i / D, k = i % D;
+      xs[e][k] = e < ne ? (double)__bfloat162float(x[(int64_t)qr[e0 + e] * D + k]) : 0.0;
+    }
     __syncthreads();
-    double bv = -INFINITY;
-    int bi = 0x7fffffff;
-    for (int j = tid; j < half; j += 128) {
-      const uint4* rr = reinterpret_cast<const uint4*>(Rt + ((int64_t)r * rows_per_round + j) * D);
-      double acc = 0.0;
+    double bv[E];
+    int bi[E];
 #pragma unroll
+    for (int e = 0; e < E; ++e) {
+      bv[e] = -INFINITY;
+      bi[e] = 0x7fffffff;
+    }
+    for (int j = tid; j < half; j += 128) {
+      const uint4* rr = reinterpret_cast<const uint4*>(Rr + (int64_t)j * D);
+      double acc[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = 0.0;
+#pragma unroll 2
       for (int c = 0; c < D / 8; ++c) {
         float f[8];
         Vec16<__nv_bfloat16>::unpack(__ldg(rr + c), f);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) acc = fma(xs[c * 8 + u], (double)f[u], acc);
+        for (int u = 0; u < 8; ++u) {
+          const double rv = (double)f[u];
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] = fma(xs[e][c * 8 + u], rv, acc[e]);
+        }
       }
-      argmax_update(acc, j, bv, bi);
-      argmax_update(-acc, half + j, bv, bi);
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        argmax_update(acc[e], j, bv[e], bi[e]);
+        argmax_update(-acc[e], half + j, bv[e], bi[e]);
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      argmax_update(ov, oi, bv, bi);
-    }
-    if (lane == 0) {
-      wv[warp] = bv;
-      wi[warp] = bi;
+    for (int e = 0; e < E; ++e) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(0xffffffffu, bv[e], o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi[e], o);
+        argmax_update(ov, oi, bv[e], bi[e]);
+      }
+      if (lane == 0) {
+        wv[warp][e] = bv[e];
+        wi[warp][e] = bi[e];
+      }
     }
     __syncthreads();
-    if (tid == 0) {
-      for (int w = 1; w < 4; ++w) argmax_update(wv[w], wi[w], bv, bi);
+    if (tid < ne) {
+      double v = wv[0][tid];
+      int b = wi[0][tid];
+      for (int w = 1; w < 4; ++w) argmax_update(wv[w][tid], wi[w][tid], v, b);
+      const int64_t row = (int64_t)qr[e0 + tid];
       const int64_t bh = row / n;
       const int t = (int)(row % n);
-      buckets[(bh * rounds + r) * n + t] = bi;
+      buckets[(bh * rounds + r) * n + t] = b;
     }
     __syncthreads();
   }
@@ -165,8 +194,9 @@ __global__ void __launch_bounds__(128)
 // ---------------------------------------------------------------------------
 struct HashTcArgs {
   int32_t* buckets;   // [BH][rounds][n]
-  uint64_t* refine;   // queue of near-tie entries
-  WsHeader* hdr;      // counters; rnorm bits in hdr->pad[0..rounds)
+  uint64_t* refine;   // near-tie queues, one of `cap` entries per round
+  int64_t cap;        // BH * n
+  WsHeader* hdr;      // rnorm bits in hdr->pad[0, 16), queue lengths in hdr->pad[16, 32)
   int n, nb, rounds, tiles_per_seq, tiles, ctas_per_group;
 };
 
@@ -419,8 +449,9 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
             const int64_t at = ((int64_t)bh * a.rounds + r) * a.n + t;
             a.buckets[at] = bucket;
             if (!(m1 - m2 > tau)) {
-              const uint32_t k = atomicAdd(&a.hdr->hash_refined, 1u);
-              a.refine[k] = ((uint64_t)((int64_t)bh * a.n + t) << 5) | (uint64_t)r;
+              atomicAdd(&a.hdr->hash_refined, 1u);
+              const uint32_t k = atomicAdd(&a.hdr->pad[16 + r], 1u);
+              a.refine[r * a.cap + k] = (uint64_t)((int64_t)bh * a.n + t);
             }
           }
         }

@@ -160,6 +160,7 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
   HashTcArgs a;
   a.buckets = buckets;
   a.refine = refine;
+  a.cap = D.BH * D.n;
   a.hdr = hdr;
   a.n = D.n;
   a.nb = D.nb;
@@ -185,12 +186,14 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
       return LSH_ERR_CUDA;
     kern<<<grid, kHashWarps * 32, p.smem, st>>>(tmx, tmr, a, p);
   }
+  dim3 rg((unsigned)((4 * sms + D.rounds - 1) / D.rounds), D.rounds);
   if (D.d == 64)
-    k_hash_refine<64><<<8 * sms, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine,
-                                               buckets, D.n, D.nb, D.rounds, rows_per_round, hdr);
+    k_hash_refine<64><<<rg, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine, a.cap,
+                                          buckets, D.n, D.nb, D.rounds, rows_per_round, hdr);
   else
-    k_hash_refine<128><<<8 * sms, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine,
-                                                buckets, D.n, D.nb, D.rounds, rows_per_round, hdr);
+    k_hash_refine<128><<<rg, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine,
+                                           a.cap, buckets, D.n, D.nb, D.rounds, rows_per_round,
+                                           hdr);
   return last_cuda();
 }
 
