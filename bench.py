@@ -36,12 +36,42 @@ METRIC = "LSH-attn fwd tokens/sec at n=64K, 4 rounds; % of HBM / tensor-pipe roo
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ("hash", "sort_gather", "chunk_attention", "unsort_merge")
+# kernels between consecutive profiling events, and the stage each belongs to
+KERNELS = lb.PROFILE_KERNELS
+KERNEL_STAGE = {"hash_prep": "hash", "hash_mma": "hash", "hash_refine": "hash",
+                "sort_hist": "sort_gather", "sort_scan": "sort_gather",
+                "sort_scatter_gather": "sort_gather", "chunk_attention": "chunk_attention",
+                "unsort_merge": "unsort_merge"}
+# the kernel that carries a stage's algorithmic work
+STAGE_KERNEL = {"hash": "hash_mma", "sort_gather": "sort_scatter_gather",
+                "chunk_attention": "chunk_attention", "unsort_merge": "unsort_merge"}
+# DRAM bytes (read + write) per launch from one ncu capture of the long-64k
+# workload, valid only while the kernel's source file is unchanged (sha256
+# of the file at capture time); see profiles/.
+NCU_TRAFFIC = {
+    "hash_prep": {"bytes": 532000, "file": "hash_tc.cuh",
+        "sha256": "fd7b1da74b7ccb46fa154ea28d82c754ea1ba45bfdd1c9d9882f40c3c4fe2ea7"},
+    "hash_mma": {"bytes": 146183000, "file": "hash_tc.cuh",
+        "sha256": "fd7b1da74b7ccb46fa154ea28d82c754ea1ba45bfdd1c9d9882f40c3c4fe2ea7"},
+    "hash_refine": {"bytes": 2043999, "file": "hash_tc.cuh",
+        "sha256": "fd7b1da74b7ccb46fa154ea28d82c754ea1ba45bfdd1c9d9882f40c3c4fe2ea7"},
+    "sort_hist": {"bytes": 8393000, "file": "sort.cuh",
+        "sha256": "78dde6d10c34979fa002a0f5e893d594535ca454bedca2ed29195ad246d2ef5a"},
+    "sort_scan": {"bytes": 2102000, "file": "sort.cuh",
+        "sha256": "78dde6d10c34979fa002a0f5e893d594535ca454bedca2ed29195ad246d2ef5a"},
+    "sort_scatter_gather": {"bytes": 1423398000, "file": "sort.cuh",
+        "sha256": "78dde6d10c34979fa002a0f5e893d594535ca454bedca2ed29195ad246d2ef5a"},
+    "chunk_attention": {"bytes": 2127058000, "file": "attn_tc.cuh",
+        "sha256": "a7fb05db1c0966392c14da11f5d33b9c4854904f9509f21acdacc187a3522449"},
+    "unsort_merge": {"bytes": 1227627000, "file": "merge.cuh",
+        "sha256": "b0c7ab1f33ff564b578073c8d8eb0b5bee9357cc6c2f8c04e8c21868a6947540"},
+}
 
 
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default=I.LONG_64K.name, choices=sorted(I.WORKLOADS))
@@ -77,48 +107,56 @@ def peaks():
 
 # ----------------------------------------------------------------------------
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while it runs."""
+    """SM clock and clock-event (throttle) reasons read through NVML every 20 ms
+    in a background thread; only samples inside [start(), stop()) count."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
-    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
 
     def __init__(self, device_index: int):
-        self.proc = None
-        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        import threading
+        self.samples, self.window, self.handle = [], None, None
+        self._stop = threading.Event()
         try:
+            import pynvml
+            pynvml.nvmlInit()
             uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", uuid], stdout=self.file, stderr=subprocess.DEVNULL)
-        except (OSError, RuntimeError):
-            self.proc = None
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
+        except Exception:  # no NVML on this host: report no samples
+            self.handle = None
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def start(self):
+        self.t0 = time.perf_counter()
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        self.proc.terminate()
-        self.proc.wait(timeout=10)
-        self.file.flush()
-        self.file.seek(0)
-        sm, smax, reasons = [], [], set()
-        for line in self.file.read().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) != 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for name, val in zip(self.NAMES, parts[3:]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        os.unlink(self.file.name)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        t1 = time.perf_counter()
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": "unavailable"}
+        self._stop.set()
+        self.thread.join(timeout=2)
+        inside = [(m, r) for (t, m, r) in self.samples if self.t0 <= t < t1]
+        reasons = sorted({name for (_, r) in inside for name, bit in self.REASONS.items()
+                          if r & bit})
+        return {"sm_mhz": statistics.median(m for m, _ in inside) if inside else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
+                "source": "NVML every 20 ms during the timed region"}
 
 
 # ----------------------------------------------------------------------------
@@ -233,7 +271,8 @@ def run_ours(args, w):
         return e
 
     K, W = args.steps, args.warmup
-    ev = [[new_event() for _ in range(5)] for _ in range(K)]
+    NE = lb.PROFILE_EVENTS
+    ev = [[new_event() for _ in range(NE)] for _ in range(K)]
     clocks = ClockSampler(local)
     for _ in range(W):
         fwd()
@@ -246,6 +285,7 @@ def run_ours(args, w):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
+    clocks.start()
     start.record(stream)
     for k in range(K):
         fwd(ev[k])
@@ -255,9 +295,11 @@ def run_ours(args, w):
     clk = clocks.stop()
     local_ms = start.elapsed_time(end)
     total_ms = max_over_ranks(local_ms, world, dev)
-    stage_ms = {}
-    for i, name in enumerate(STAGES):
-        stage_ms[name] = statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(K))
+    kernel_ms = {}
+    for i, name in enumerate(KERNELS):
+        kernel_ms[name] = statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(K))
+    stage_ms = {st: sum(t for kn, t in kernel_ms.items() if KERNEL_STAGE[kn] == st)
+                for st in STAGES}
     value = world * w.tokens * K / (total_ms / 1e3)
 
     # ---- end to end through the public API: pinned host in, host out
@@ -292,29 +334,35 @@ def run_ours(args, w):
         return
     alg = algorithmic(w)
     pk, pk_kind = peaks()
-    dom = max(STAGES, key=lambda s: stage_ms[s])
     timed_s = total_ms / 1e3
-    tensor_bound = {"hash": w.n_buckets // 2 >= 256, "chunk_attention": False}
     stages = {}
-    for s in STAGES:
-        t = stage_ms[s] / 1e3
-        gbs = alg[s]["bytes"] / t / 1e9
-        tfs = alg[s]["flops"] / t / 1e12
-        stages[s] = {"ms": round(stage_ms[s], 4), "GB/s": round(gbs, 1),
-                     "hbm_frac": round(gbs / pk["hbm_gbs"], 4),
-                     "TFLOP/s": round(tfs, 2)}
-    if tensor_bound.get(dom, False):
+    for st in STAGES:
+        t = stage_ms[st] / 1e3
+        stages[st] = {"ms": round(stage_ms[st], 4),
+                      "GB/s": round(alg[st]["bytes"] / t / 1e9, 1),
+                      "hbm_frac": round(alg[st]["bytes"] / t / 1e9 / pk["hbm_gbs"], 4),
+                      "TFLOP/s": round(alg[st]["flops"] / t / 1e12, 2)}
+    kernels = {kn: round(t, 4) for kn, t in kernel_ms.items()}
+    # roofline of the dominant kernel, against its own launch time
+    dom = max(KERNELS, key=lambda kn: kernel_ms[kn])
+    dst = KERNEL_STAGE[dom]
+    dsec = kernel_ms[dom] / 1e3
+    carries = STAGE_KERNEL[dst] == dom
+    tensor = dst in ("hash", "chunk_attention") and alg[dst]["flops"] / max(1, alg[dst]["bytes"]) > \
+        1e3 * pk["bf16_tflops"] / pk["hbm_gbs"]
+    if carries and tensor:
         peak = pk["bf16_tflops_sustained"] if timed_s > 1.0 else pk["bf16_tflops"]
-        achieved = alg[dom]["flops"] / (stage_ms[dom] / 1e3) / 1e12
-        roof = {"bound": "tensor", "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "unit": "TFLOP/s",
+                "achieved": round(alg[dst]["flops"] / dsec / 1e12, 2), "peak": peak}
     else:
-        peak = pk["hbm_gbs"]
-        achieved = alg[dom]["bytes"] / (stage_ms[dom] / 1e3) / 1e9
-        roof = {"bound": "hbm", "unit": "GB/s"}
-    roof.update({"kernel": dom, "achieved": round(achieved, 2), "peak": peak,
-                 "frac": round(achieved / peak, 4), "traffic": None,
-                 "peak_source": f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured"
-                 else "fallback"})
+        roof = {"bound": "hbm", "unit": "GB/s",
+                "achieved": round((alg[dst]["bytes"] if carries else 0) / dsec / 1e9, 1),
+                "peak": pk["hbm_gbs"]}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["kernel"] = dom
+    roof["traffic"] = traffic_of(dom)
+    roof["peak_source"] = "of measured (MEASURED_PEAKS.json)" if pk_kind == "measured" else \
+        "of fallback"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
@@ -325,8 +373,8 @@ def run_ours(args, w):
         "gpu_launches": K * launches_per_forward(buckets_given=False),
         "roofline": roof,
         "stages": stages,
-        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"],
-                   "reasons": clk["reasons"], "samples": clk["samples"]},
+        "kernels_ms": kernels,
+        "clocks": clk,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
@@ -334,8 +382,22 @@ def run_ours(args, w):
 
 
 def launches_per_forward(buckets_given: bool) -> int:
-    # hash (1) + sort: histogram, scan, rank/scatter/gather (3) + attention (1) + merge (1)
-    return (0 if buckets_given else 1) + 3 + 1 + 1
+    # hash: rotation transpose, projection/argmax, fp64 re-decision (3); sort:
+    # histogram, scan, rank/scatter/gather (3); attention (1); merge (1)
+    return (0 if buckets_given else 3) + 3 + 1 + 1
+
+
+def traffic_of(kernel: str):
+    """ncu DRAM bytes per launch of `kernel`, if its source is unchanged."""
+    import hashlib
+    rec = NCU_TRAFFIC.get(kernel)
+    if rec is None:
+        return None
+    path = os.path.join(ROOT, "lsh_attention_b200", "csrc", rec["file"])
+    with open(path, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+            return None
+    return rec["bytes"]
 
 
 def main():

@@ -123,12 +123,20 @@ lsh_status lsh_attn_forward(const lsh_attn_desc *desc, const void *x, const void
                             const void *R, const int32_t *buckets, void *out, float *lse,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/* Number of events lsh_attn_forward_profiled records. */
+#define LSH_ATTN_PROFILE_EVENTS 9
+
 /* lsh_attn_forward that also records the caller's CUDA events on `stream`
- * at the stage boundaries, for timing each stage on the device:
- *   events[0] before the hash      events[1] after the hash (right after
- *   events[0] when buckets are given)   events[2] after the sort and gather
- *   events[3] after the chunked attention   events[4] after the round merge.
- * `events` points to 5 cudaEvent_t handles created by the caller. */
+ * at every kernel boundary, for timing each kernel on the device:
+ *   [0] start               [1] after the rotation transpose of the hash
+ *   [2] after the projection / argmax kernel  [3] after the fp64 re-decision
+ *   [4] after the bucket histograms  [5] after their scan
+ *   [6] after the stable ranks, perm/inv and row gather
+ *   [7] after the chunked attention  [8] after the un-sort and round merge
+ * A kernel that does not run for this problem (caller-supplied buckets, the
+ * fp64 hash) leaves consecutive events with nothing between them.
+ * `events` points to LSH_ATTN_PROFILE_EVENTS cudaEvent_t handles created by
+ * the caller. */
 lsh_status lsh_attn_forward_profiled(const lsh_attn_desc *desc, const void *x, const void *v,
                                      const void *R, const int32_t *buckets, void *out, float *lse,
                                      void *workspace, size_t workspace_bytes, void *stream,

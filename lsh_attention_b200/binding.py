@@ -16,6 +16,10 @@ import torch
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblshattn.so")
 
 LSH_F32, LSH_BF16 = 0, 1
+PROFILE_EVENTS = 9  # LSH_ATTN_PROFILE_EVENTS
+#: what ends at each profiling event after the first
+PROFILE_KERNELS = ("hash_prep", "hash_mma", "hash_refine", "sort_hist", "sort_scan",
+                   "sort_scatter_gather", "chunk_attention", "unsort_merge")
 _DTYPES = {torch.float32: LSH_F32, torch.bfloat16: LSH_BF16}
 
 #: every symbol the header declares
@@ -184,8 +188,9 @@ def lsh_attn_forward(x, v, R=None, *, n_buckets: int, chunk: int, causal: bool, 
                      buckets=None, out=None, lse=None, ws=None, stream=None, events=None):
     """LSH-attention forward. x, v [B, H, n, d]; R [rounds, d, nb/2] (or
     caller buckets [B, H, rounds, n]). Returns (out [B, H, n, d], lse
-    [B, H, rounds, n] fp32). `events`: five recorded torch.cuda.Event objects
-    to mark the stage boundaries (lsh_attn_forward_profiled)."""
+    [B, H, rounds, n] fp32). `events`: PROFILE_EVENTS recorded
+    torch.cuda.Event objects marking the kernel boundaries
+    (lsh_attn_forward_profiled)."""
     B, H, n, d = x.shape
     _require(x, "x", None, None)
     _require(v, "v", x.dtype, tuple(x.shape))
@@ -211,9 +216,9 @@ def lsh_attn_forward(x, v, R=None, *, n_buckets: int, chunk: int, causal: bool, 
     if events is None:
         _check(load().lsh_attn_forward(*args))
     else:
-        if len(events) != 5 or any(e.cuda_event == 0 for e in events):
-            raise ValueError("events: five torch.cuda.Event objects, each recorded once")
-        ev = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+        if len(events) != PROFILE_EVENTS or any(e.cuda_event == 0 for e in events):
+            raise ValueError(f"events: {PROFILE_EVENTS} torch.cuda.Event objects, each recorded once")
+        ev = (ctypes.c_void_p * PROFILE_EVENTS)(*[e.cuda_event for e in events])
         _check(load().lsh_attn_forward_profiled(*args, ev))
     return out, lse
 

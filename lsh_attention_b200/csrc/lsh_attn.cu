@@ -113,6 +113,14 @@ lsh_status reset_header(void* ws, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------- launches
+// Profiling marks: the events of lsh_attn_forward_profiled, one per kernel
+// boundary (indices in lsh_attn.h).
+inline lsh_status mark(void* const* events, int i, cudaStream_t st) {
+  if (!events) return LSH_OK;
+  return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess ? LSH_OK
+                                                                              : LSH_ERR_CUDA;
+}
+
 lsh_status launch_hash_exact(const Dims& D, const void* x, const void* R, int32_t* buckets,
                              cudaStream_t st, bool bf16) {
   const int esz = bf16 ? 2 : 4;
@@ -142,9 +150,15 @@ lsh_status launch_hash_exact(const Dims& D, const void* x, const void* R, int32_
 
 // bf16: tcgen05 projection + top-2 screen, fp64 re-decision of near ties.
 lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const void* R,
-                          int32_t* buckets, void* ws, cudaStream_t st) {
+                          int32_t* buckets, void* ws, cudaStream_t st, void* const* ev) {
   const HashTcPlan p = hash_tc_plan(D.d, D.nb, D.rounds);
-  if (p.group == 0) return launch_hash_exact(D, x, R, buckets, st, true);
+  lsh_status s;
+  if (p.group == 0) {
+    if ((s = mark(ev, 1, st)) != LSH_OK) return s;
+    if ((s = launch_hash_exact(D, x, R, buckets, st, true)) != LSH_OK) return s;
+    if ((s = mark(ev, 2, st)) != LSH_OK) return s;
+    return mark(ev, 3, st);
+  }
   WsHeader* hdr = at<WsHeader>(ws, L.header);
   __nv_bfloat16* rt = at<__nv_bfloat16>(ws, L.rt);
   uint64_t* refine = at<uint64_t>(ws, L.refine);
@@ -152,6 +166,7 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
   dim3 pg((rows_per_round + 31) / 32, D.rounds);
   k_hash_prep<<<pg, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(R), rt, hdr->pad, D.d, p.half,
                                   rows_per_round);
+  if ((s = mark(ev, 1, st)) != LSH_OK) return s;
   CUtensorMap tmx, tmr;
   if (!make_tmap_bf16_2d(&tmx, x, D.d, (uint64_t)D.BH * D.n, (uint64_t)D.d * 2, 64, kHashTile) ||
       !make_tmap_bf16_2d(&tmr, rt, D.d, (uint64_t)D.rounds * rows_per_round, (uint64_t)D.d * 2, 64,
@@ -186,6 +201,7 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
       return LSH_ERR_CUDA;
     kern<<<grid, kHashWarps * 32, p.smem, st>>>(tmx, tmr, a, p);
   }
+  if ((s = mark(ev, 2, st)) != LSH_OK) return s;
   dim3 rg((unsigned)((4 * sms + D.rounds - 1) / D.rounds), D.rounds);
   if (D.d == 64)
     k_hash_refine<64><<<rg, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine, a.cap,
@@ -194,24 +210,32 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
     k_hash_refine<128><<<rg, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine,
                                            a.cap, buckets, D.n, D.nb, D.rounds, rows_per_round,
                                            hdr);
-  return last_cuda();
+  if ((s = last_cuda()) != LSH_OK) return s;
+  return mark(ev, 3, st);
 }
 
 lsh_status launch_hash(const Dims& D, const Layout& L, const void* x, const void* R,
-                       int32_t* buckets, void* ws, cudaStream_t st) {
-  if (D.dtype == LSH_BF16) return launch_hash_tc(D, L, x, R, buckets, ws, st);
-  return launch_hash_exact(D, x, R, buckets, st, false);
+                       int32_t* buckets, void* ws, cudaStream_t st, void* const* ev = nullptr) {
+  if (D.dtype == LSH_BF16) return launch_hash_tc(D, L, x, R, buckets, ws, st, ev);
+  lsh_status s;
+  if ((s = mark(ev, 1, st)) != LSH_OK) return s;
+  if ((s = launch_hash_exact(D, x, R, buckets, st, false)) != LSH_OK) return s;
+  if ((s = mark(ev, 2, st)) != LSH_OK) return s;
+  return mark(ev, 3, st);
 }
 
 template <typename T>
 lsh_status launch_sort(const Dims& D, const int32_t* buckets, const void* x, const void* v,
                        int32_t* perm, int32_t* inv, void* xs, void* vs, float* invnorm,
-                       int32_t* hist, WsHeader* hdr, cudaStream_t st) {
+                       int32_t* hist, WsHeader* hdr, cudaStream_t st, void* const* ev = nullptr) {
+  lsh_status s;
   const int tile = sort_tile(D.nb);
   dim3 grid(D.tiles, (unsigned)D.S);
   k_sort_hist<<<grid, 256, sizeof(int32_t) * D.nb, st>>>(buckets, D.n, D.nb, tile, D.tiles, hist,
                                                          hdr);
+  if ((s = mark(ev, 4, st)) != LSH_OK) return s;
   k_sort_scan<<<(unsigned)D.S, 1024, 0, st>>>(hist, D.nb * D.tiles);
+  if ((s = mark(ev, 5, st)) != LSH_OK) return s;
   const int nw = sort_warps(D.nb);
   const size_t smem = sizeof(int32_t) * (size_t)nw * D.nb;
   auto kern = k_sort_scatter<T>;
@@ -222,7 +246,8 @@ lsh_status launch_sort(const Dims& D, const int32_t* buckets, const void* x, con
                                      static_cast<const T*>(v), perm, inv, static_cast<T*>(xs),
                                      static_cast<T*>(vs), invnorm, D.n, D.d, D.nb, D.rounds,
                                      D.tiles);
-  return last_cuda();
+  if ((s = last_cuda()) != LSH_OK) return s;
+  return mark(ev, 6, st);
 }
 
 template <typename T, int DD, int QPW>
@@ -307,13 +332,6 @@ lsh_status launch_merge(const Dims& D, const int32_t* inv, const float* lse_s, c
   return last_cuda();
 }
 
-// Record events[i] (if any) on the stream.
-inline lsh_status mark(void* const* events, int i, cudaStream_t st) {
-  if (!events) return LSH_OK;
-  return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), st) == cudaSuccess ? LSH_OK
-                                                                              : LSH_ERR_CUDA;
-}
-
 template <typename T>
 lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const void* v,
                          const void* R, const int32_t* buckets, void* out, float* lse, void* ws,
@@ -323,10 +341,12 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
   if ((s = mark(ev, 0, st)) != LSH_OK) return s;
   if (!buckets) {
     int32_t* bk = at<int32_t>(ws, L.buckets);
-    if ((s = launch_hash(D, L, x, R, bk, ws, st)) != LSH_OK) return s;
+    if ((s = launch_hash(D, L, x, R, bk, ws, st, ev)) != LSH_OK) return s;
     buckets = bk;
+  } else {
+    for (int i = 1; i <= 3; ++i)
+      if ((s = mark(ev, i, st)) != LSH_OK) return s;
   }
-  if ((s = mark(ev, 1, st)) != LSH_OK) return s;
   int32_t* perm = at<int32_t>(ws, L.perm);
   int32_t* inv = at<int32_t>(ws, L.inv);
   float* invnorm = at<float>(ws, L.invnorm);
@@ -335,20 +355,19 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
   float* out_s = at<float>(ws, L.out_s);
   float* lse_s = at<float>(ws, L.lse_s);
   if ((s = launch_sort<T>(D, buckets, x, v, perm, inv, xs, vs, invnorm, at<int32_t>(ws, L.hist),
-                          hdr, st)) != LSH_OK)
+                          hdr, st, ev)) != LSH_OK)
     return s;
-  if ((s = mark(ev, 2, st)) != LSH_OK) return s;
   if (attn_tc_supported(D))
     s = launch_attn_tc(D, xs, vs, perm, invnorm, out_s, lse_s, hdr, st);
   else
     s = D.d == 64 ? launch_attn_simt<T, 64>(D, xs, vs, perm, invnorm, out_s, lse_s, st)
                   : launch_attn_simt<T, 128>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
   if (s != LSH_OK) return s;
-  if ((s = mark(ev, 3, st)) != LSH_OK) return s;
+  if ((s = mark(ev, 7, st)) != LSH_OK) return s;
   s = D.d == 64 ? launch_merge<T, 64>(D, inv, lse_s, out_s, out, lse, st)
                 : launch_merge<T, 128>(D, inv, lse_s, out_s, out, lse, st);
   if (s != LSH_OK) return s;
-  return mark(ev, 4, st);
+  return mark(ev, 8, st);
 }
 
 }  // namespace

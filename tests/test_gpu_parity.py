@@ -358,3 +358,23 @@ def test_hash_refine_count_is_small():
     print(f"{w.name}: {diag['hash_refined']} of {total} hashes re-decided in fp64")
     assert diag["status"] == 0
     assert 0 < diag["hash_refined"] < 0.02 * total
+
+
+def test_profiled_forward_matches_and_times_every_kernel():
+    w = I.BF16_SHORT
+    x, v = I.make_qkv(w)
+    R = I.make_rotations(w)
+    xg, vg, Rg = to_gpu(x, v, R)
+    kw = dict(n_buckets=w.n_buckets, chunk=w.chunk, causal=w.causal)
+    ref = [t.clone() for t in lb.lsh_attn_forward(xg, vg, Rg, **kw)]
+    evs = []
+    for _ in range(lb.PROFILE_EVENTS):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        evs.append(e)
+    out, lse = lb.lsh_attn_forward(xg, vg, Rg, events=evs, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1])
+    times = [evs[i].elapsed_time(evs[i + 1]) for i in range(lb.PROFILE_EVENTS - 1)]
+    assert all(t >= 0 for t in times)
+    assert times[1] > 0 and times[6] > 0  # projection kernel, attention kernel
