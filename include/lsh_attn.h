@@ -149,6 +149,31 @@ lsh_status lsh_attn_get_device_status(const void *workspace, void *stream);
 /* Synchronise `stream` and copy the workspace counters into *diag. */
 lsh_status lsh_attn_get_diag(const void *workspace, void *stream, lsh_attn_diag *diag);
 
+/* Size of the device-resident scratch of lsh_attn_sort_noalloc (8 MiB). */
+#define LSH_ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* The stable sort of lsh_attn_sort (perm only, no row gather) for callers
+ * that must not allocate device memory and cannot pass a workspace: for
+ * example a plug-in whose host runtime owns all device memory, or a loop that
+ * cannot afford the device synchronisation of cudaMalloc / cudaFree. The
+ * paper has no counterpart to this entry point; it only changes where the
+ * scratch lives. No memory is allocated: the scratch is a fixed array of
+ * LSH_ATTN_NOALLOC_SCRATCH_BYTES in the library's own device memory, held by
+ * every GPU that loads the library until the process exits.
+ *   - buckets [B][H][Rn][n] int32 in; perm [B][H][Rn][n] int32 out (device).
+ *   - A problem needs 256 + 4*B*H*Rn*nb*ceil(n / T) (rounded up to 256) +
+ *     4*B*H*Rn*n bytes of scratch, T = 256 * clamp(16384 / nb, 1, 16); larger
+ *     problems return LSH_ERR_UNSUPPORTED and write nothing (use lsh_attn_sort).
+ *   - The first call on a device looks up the scratch's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one scratch, whose contents persist
+ *     from the previous call: calls that may overlap on the GPU (different
+ *     streams without ordering between them) race and must not be issued.
+ *   - Errors as for lsh_attn_sort; kernel-side status is not readable here. */
+lsh_status lsh_attn_sort_noalloc(const lsh_attn_desc *desc, const int32_t *buckets,
+                                 int32_t *perm, void *stream);
+
 /* Static, human-readable name of a status code. */
 const char *lsh_attn_status_string(lsh_status status);
 

@@ -25,7 +25,7 @@ _DTYPES = {torch.float32: LSH_F32, torch.bfloat16: LSH_BF16}
 #: every symbol the header declares
 EXPORTS = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_forward",
            "lsh_attn_forward_profiled", "lsh_attn_get_device_status", "lsh_attn_get_diag",
-           "lsh_attn_status_string")
+           "lsh_attn_sort_noalloc", "lsh_attn_status_string")
 
 
 class LshAttnDesc(ctypes.Structure):
@@ -70,6 +70,7 @@ def load() -> ctypes.CDLL:
             lib.lsh_attn_forward_profiled.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
                                                       ctypes.POINTER(ctypes.c_void_p)]
             lib.lsh_attn_get_device_status.argtypes = [vp, vp]
+            lib.lsh_attn_sort_noalloc.argtypes = [dp, vp, vp, vp]
             lib.lsh_attn_get_diag.argtypes = [vp, vp, ctypes.POINTER(LshAttnDiag)]
             lib.lsh_attn_status_string.argtypes = [ctypes.c_int]
             lib.lsh_attn_status_string.restype = ctypes.c_char_p
@@ -221,6 +222,20 @@ def lsh_attn_forward(x, v, R=None, *, n_buckets: int, chunk: int, causal: bool, 
         ev = (ctypes.c_void_p * PROFILE_EVENTS)(*[e.cuda_event for e in events])
         _check(load().lsh_attn_forward_profiled(*args, ev))
     return out, lse
+
+
+def lsh_attn_sort_noalloc(buckets, n_buckets: int, perm=None, stream=None):
+    """perm [B, H, rounds, n] of the stable bucket sort without any workspace:
+    the library's fixed device scratch is used (see lsh_attn.h)."""
+    B, H, rounds, n = buckets.shape
+    _require(buckets, "buckets", torch.int32, None)
+    desc = make_desc(B, H, n, 64, n_buckets, 1, rounds, False, torch.bfloat16)
+    if perm is None:
+        perm = torch.empty((B, H, rounds, n), dtype=torch.int32, device=buckets.device)
+    _require(perm, "perm", torch.int32, (B, H, rounds, n))
+    _check(load().lsh_attn_sort_noalloc(ctypes.byref(desc), _ptr(buckets), _ptr(perm),
+                                        _stream(stream)))
+    return perm
 
 
 def lsh_attn_get_diag(ws, stream=None) -> dict:

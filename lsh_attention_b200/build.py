@@ -36,7 +36,7 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
         return LIB
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + \
-        ["-o", tmp, os.path.join(CSRC, "lsh_attn.cu")]
+        ["-o", tmp, os.path.join(CSRC, "lsh_attn.cu"), os.path.join(CSRC, "lsh_attn_noalloc.cu")]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB
