@@ -25,7 +25,8 @@
 //               self logit) is flagged: its output is v of the query itself.
 //   warps 6..9  epilogue: O from TMEM, divided by the row sum, staged per warp
 //               in a 4 KB swizzled buffer (32 rows x 32 fp32) and written by
-//               TMA bulk stores, so every 128-byte line leaves the SM whole
+//               TMA bulk stores (slot order), so every 128-byte line leaves the
+//               SM whole; the softmax writes lse at the query's position
 // TMEM: S[0] = [0, 192), S[1] = [192, 384), O = [384, 384 + d).
 #pragma once
 
@@ -46,8 +47,8 @@ struct AttnTcArgs {
   const float* invnorm;        // [S][n] 1/||x|| of the sorted rows (0 for a zero row)
   const int32_t* perm;         // [S][n] position of each slot
   const __nv_bfloat16* vs;     // [S][n][d] sorted v rows (self-only rows copy theirs)
-  float* out_s;                // [S][n][d] fp32, slot order
-  float* lse_s;                // [S][n]
+  float* out_r;                // [S][n][d] fp32, each round's output in slot order
+  float* lse;                  // [S][n] each round's lse by position (the caller's output)
   WsHeader* hdr;
   int n, causal, pairs_per_seg;
   int64_t pairs;               // S * pairs_per_seg
@@ -78,7 +79,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   float* kinv = reinterpret_cast<float*>(ostage + 4 * 32 * 128);     // [2][192]
   int32_t* kpos = reinterpret_cast<int32_t*>(kinv + 2 * kAttnKeys);  // [2][192]
   float2* ktab = reinterpret_cast<float2*>(kpos + 2 * kAttnKeys);    // [2][192] (scale, pos)
-  float* rstat = reinterpret_cast<float*>(ktab + 2 * kAttnKeys);     // [4][128]
+  float* rstat = reinterpret_cast<float*>(ktab + 2 * kAttnKeys);     // [4][128] 1/sum
   uint64_t* bars = reinterpret_cast<uint64_t*>(rstat + kAttnStats * 128);
   uint64_t* xfull = bars + 0;    // [2] tx: x tile + metadata
   uint64_t* xfree = bars + 2;    // [2] S MMA done + 4 softmax warps done with the metadata
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       // lse over the visible keys and the self logit; exp(-1e5) vanishes
       // unless the row sees nothing else
       if (qs < a.n)
-        a.lse_s[seg * a.n + qs] = sum > 0.f ? (bound + log2f(sum)) * 0.6931471805599453f
+        a.lse[seg * a.n + qpos] = sum > 0.f ? (bound + log2f(sum)) * 0.6931471805599453f
                                             : kSelfLogit;
       rstat[(i % kAttnStats) * 128 + row] = sum > 0.f ? 1.0f / sum : -1.f;
       tc_fence_before();

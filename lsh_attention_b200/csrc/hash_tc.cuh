@@ -10,8 +10,10 @@
 //   * warp 1 issues tcgen05.mma (M = 128 tokens, N <= 256 columns, K = d)
 //     into one of two TMEM accumulators, so the next unit's MMA overlaps the
 //     epilogue of the current one;
-//   * warps 2..9 read the fp32 projections with tcgen05.ld and keep, per
-//     token, the largest and second largest |p_j|, the argmax and its sign.
+//   * warps 2..13 read the fp32 projections with tcgen05.ld and keep, per
+//     token, the largest and second largest |p_j|, the argmax and its sign
+//     (three warps per TMEM lane quadrant, each on every third 16-column
+//     batch).
 // Exactness: the fp32 accumulation of d bf16 products is within
 // d * 2^-23 * sum_k |x_k R_kj| <= d * 2^-23 * ||x|| ||R_j|| of the exact sum,
 // whatever the order or rounding of the additions. When the top two |p| are
@@ -28,7 +30,8 @@ namespace lsh {
 
 constexpr int kHashTile = 128;       // tokens per tile (MMA M)
 constexpr int kHashMaxN = 256;       // columns per MMA (N)
-constexpr int kHashWarps = 10;       // 0: TMA, 1: MMA, 2..9: epilogue
+constexpr int kHashEpiPerQuad = 3;   // epilogue warps per TMEM lane quadrant
+constexpr int kHashWarps = 2 + 4 * kHashEpiPerQuad;  // 0: TMA, 1: MMA, rest: epilogue
 constexpr float kTieFactor = 4.0f;   // margin threshold / accumulation error bound
 constexpr int kHashSmemBudget = 227 * 1024;
 
@@ -53,7 +56,7 @@ inline HashTcPlan hash_tc_plan(int d, int nb, int rounds) {
   p.ch = (p.half + p.nc - 1) / p.nc;
   p.x_bytes = (size_t)2 * p.kh * kHashTile * 128;
   const size_t per_round = (size_t)p.ch * p.kh * p.nc * 128;
-  const size_t misc = 1024 /* alignment */ + 8192 /* barriers, combine buffers */;
+  const size_t misc = 1024 /* alignment */ + 16384 /* barriers, combine buffers */;
   const size_t avail = kHashSmemBudget > (long)(p.x_bytes + misc)
                            ? kHashSmemBudget - p.x_bytes - misc
                            : 0;
@@ -254,7 +257,7 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
   uint64_t* acc_empty = bars + 7;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
-  float4* comb = reinterpret_cast<float4*>(bars + 16);  // [2][4][32]
+  float4* comb = reinterpret_cast<float4*>(bars + 16);  // [2][4][2][32]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x / a.ctas_per_group;
@@ -268,7 +271,7 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
       mbar_init(x_full + i, 1);
       mbar_init(x_empty + i, 1 + 4);  // MMA commit + 4 norm-reading warps
       mbar_init(acc_full + i, 1);
-      mbar_init(acc_empty + i, 8);    // 8 epilogue warps
+      mbar_init(acc_empty + i, 4 * kHashEpiPerQuad);  // every epilogue warp
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
     // ------------------------------------------------------------ epilogue
     const int e = warp - 2;
     const int q = warp & 3;       // TMEM lane quadrant this warp may access
-    const int h = e >> 2;         // column-batch parity handled by this warp
+    const int h = e >> 2;         // this warp takes the 16-column batches b = h (mod 3)
     const int row = q * 32 + lane;
     const uint32_t tlane = (uint32_t)(q * 32) << 16;
     const float* rnorm = reinterpret_cast<const float*>(a.hdr->pad);
@@ -399,17 +402,18 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
           }
           tc_fence_after();
           const uint32_t tbase = tmem + tlane + ab * p.tmem_cols;
-          // this warp's 16-column batches are h, h + 2, ...: four loads in
+          // this warp's 16-column batches are h, h + 3, ...: two loads in
           // flight per wait
-          for (int i0 = 0; 2 * i0 + h < nbatch; i0 += 4) {
-            uint32_t v[4][16];
+          constexpr int P = kHashEpiPerQuad;
+          for (int i0 = 0; P * i0 + h < nbatch; i0 += 2) {
+            uint32_t v[2][16];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              if (h + 2 * (i0 + i) < nbatch) tmem_ld16(tbase + (h + 2 * (i0 + i)) * 16, v[i]);
+            for (int i = 0; i < 2; ++i)
+              if (h + P * (i0 + i) < nbatch) tmem_ld16(tbase + (h + P * (i0 + i)) * 16, v[i]);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int b = h + 2 * (i0 + i);
+            for (int i = 0; i < 2; ++i) {
+              const int b = h + P * (i0 + i);
               if (b < nbatch) {
                 const int j0 = c * p.nc + b * 16;
                 if (j0 + 16 <= p.half) {
@@ -431,15 +435,19 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
         }
 #pragma unroll
         for (int i = 1; i < kHashLanesIlp; ++i) st[0].merge(st[i].m1, st[i].m2, st[i].idx, st[i].sv);
-        // combine the two warps of this quadrant, then decide
-        float4* slot = comb + ((rc & 1) * 4 + q) * 32 + lane;
-        if (h == 1) *slot = make_float4(st[0].m1, st[0].m2, __int_as_float(st[0].idx), st[0].sv);
-        asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+        // combine the warps of this quadrant, then decide
+        float4* slot = comb + (((rc & 1) * 4 + q) * (kHashEpiPerQuad - 1)) * 32 + lane;
+        if (h > 0)
+          slot[(h - 1) * 32] = make_float4(st[0].m1, st[0].m2, __int_as_float(st[0].idx), st[0].sv);
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kHashEpiPerQuad) : "memory");
         stop = *abort_flag != 0;
         if (stop) break;
         if (h == 0) {
-          const float4 o = *slot;
-          st[0].merge(o.x, o.y, __float_as_int(o.z), o.w);
+#pragma unroll
+          for (int o_ = 0; o_ < kHashEpiPerQuad - 1; ++o_) {
+            const float4 o = slot[o_ * 32];
+            st[0].merge(o.x, o.y, __float_as_int(o.z), o.w);
+          }
           const float m1 = st[0].m1, m2 = st[0].m2, sv = st[0].sv;
           const int idx = st[0].idx;
           if (t < a.n) {

@@ -13,6 +13,7 @@
 #include "hash_tc.cuh"
 #include "merge.cuh"
 #include "sort.cuh"
+#include "sort_tma.cuh"
 #include "tma_host.cuh"
 
 namespace {
@@ -236,16 +237,32 @@ lsh_status launch_sort(const Dims& D, const int32_t* buckets, const void* x, con
   if ((s = mark(ev, 4, st)) != LSH_OK) return s;
   k_sort_scan<<<(unsigned)D.S, 1024, 0, st>>>(hist, D.nb * D.tiles);
   if ((s = mark(ev, 5, st)) != LSH_OK) return s;
-  const int nw = sort_warps(D.nb);
-  const size_t smem = sizeof(int32_t) * (size_t)nw * D.nb;
-  auto kern = k_sort_scatter<T>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return LSH_ERR_CUDA;
-  kern<<<grid, nw * 32, smem, st>>>(buckets, hist, static_cast<const T*>(x),
-                                     static_cast<const T*>(v), perm, inv, static_cast<T*>(xs),
-                                     static_cast<T*>(vs), invnorm, D.n, D.d, D.nb, D.rounds,
-                                     D.tiles);
+  if (xs != nullptr) {  // ranks + row gather, rows streamed by TMA
+    const SortGatherPlan gp = sort_gather_plan(D.nb, D.d, (int)sizeof(T));
+    CUtensorMap tmx, tmv;
+    const uint64_t rows = (uint64_t)D.BH * D.n;
+    if (!make_tmap_plain_2d(&tmx, x, (int)sizeof(T), D.d, rows, D.d, gp.chunk_rows) ||
+        !make_tmap_plain_2d(&tmv, v, (int)sizeof(T), D.d, rows, D.d, gp.chunk_rows))
+      return LSH_ERR_CUDA;
+    auto kern = k_sort_gather_tma<T>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gp.smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, gp.nw * 32, gp.smem, st>>>(tmx, tmv, buckets, hist, perm, inv,
+                                             static_cast<T*>(xs), static_cast<T*>(vs), invnorm,
+                                             D.n, D.d, D.nb, D.rounds, D.tiles, gp.chunk_rows, hdr);
+  } else {  // ranks only
+    const int nw = sort_warps(D.nb);
+    const size_t smem = sizeof(int32_t) * (size_t)nw * D.nb;
+    auto kern = k_sort_scatter<T>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, nw * 32, smem, st>>>(buckets, hist, static_cast<const T*>(x),
+                                       static_cast<const T*>(v), perm, inv, static_cast<T*>(xs),
+                                       static_cast<T*>(vs), invnorm, D.n, D.d, D.nb, D.rounds,
+                                       D.tiles);
+  }
   if ((s = last_cuda()) != LSH_OK) return s;
   return mark(ev, 6, st);
 }
@@ -292,20 +309,20 @@ lsh_status launch_attn_tc_k(const CUtensorMap& tmx, const CUtensorMap& tmv,
 }
 
 lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
-                          const float* invnorm, float* out_s, float* lse_s, WsHeader* hdr,
+                          const float* invnorm, float* out_r, float* lse, WsHeader* hdr,
                           cudaStream_t st) {
   CUtensorMap tmx, tmv, tmo;
   const uint64_t rows = (uint64_t)D.S * D.n;
   if (!make_tmap_bf16_2d(&tmx, xs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys) ||
       !make_tmap_bf16_2d(&tmv, vs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys) ||
-      !make_tmap_f32_2d(&tmo, out_s, D.d, rows, (uint64_t)D.d * 4, 32, 32))
+      !make_tmap_f32_2d(&tmo, out_r, D.d, rows, (uint64_t)D.d * 4, 32, 32))
     return LSH_ERR_CUDA;
   AttnTcArgs a;
   a.invnorm = invnorm;
   a.perm = perm;
   a.vs = static_cast<const __nv_bfloat16*>(vs);
-  a.out_s = out_s;
-  a.lse_s = lse_s;
+  a.out_r = out_r;
+  a.lse = lse;
   a.hdr = hdr;
   a.n = D.n;
   a.causal = D.causal;
@@ -323,12 +340,12 @@ lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const i
 }
 
 template <typename T, int DD>
-lsh_status launch_merge(const Dims& D, const int32_t* inv, const float* lse_s, const float* out_s,
-                        void* out, float* lse, cudaStream_t st) {
+lsh_status launch_merge(const Dims& D, const int32_t* inv, const float* lse, const float* out_r,
+                        void* out, cudaStream_t st) {
   const int64_t total = D.BH * D.n;
   const unsigned blocks = (unsigned)((total + kMergeWarps - 1) / kMergeWarps);
-  k_merge<T, DD><<<blocks, kMergeWarps * 32, 0, st>>>(inv, lse_s, out_s, static_cast<T*>(out),
-                                                        lse, D.n, D.rounds, total);
+  k_merge<T, DD><<<blocks, kMergeWarps * 32, 0, st>>>(inv, lse, out_r, static_cast<T*>(out), D.n,
+                                                        D.rounds, total);
   return last_cuda();
 }
 
@@ -352,20 +369,19 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
   float* invnorm = at<float>(ws, L.invnorm);
   void* xs = at<unsigned char>(ws, L.xs);
   void* vs = at<unsigned char>(ws, L.vs);
-  float* out_s = at<float>(ws, L.out_s);
-  float* lse_s = at<float>(ws, L.lse_s);
+  float* out_r = at<float>(ws, L.out_s);  // each round's output rows, slot order
   if ((s = launch_sort<T>(D, buckets, x, v, perm, inv, xs, vs, invnorm, at<int32_t>(ws, L.hist),
                           hdr, st, ev)) != LSH_OK)
     return s;
   if (attn_tc_supported(D))
-    s = launch_attn_tc(D, xs, vs, perm, invnorm, out_s, lse_s, hdr, st);
+    s = launch_attn_tc(D, xs, vs, perm, invnorm, out_r, lse, hdr, st);
   else
-    s = D.d == 64 ? launch_attn_simt<T, 64>(D, xs, vs, perm, invnorm, out_s, lse_s, st)
-                  : launch_attn_simt<T, 128>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
+    s = D.d == 64 ? launch_attn_simt<T, 64>(D, xs, vs, perm, invnorm, out_r, lse, st)
+                  : launch_attn_simt<T, 128>(D, xs, vs, perm, invnorm, out_r, lse, st);
   if (s != LSH_OK) return s;
   if ((s = mark(ev, 7, st)) != LSH_OK) return s;
-  s = D.d == 64 ? launch_merge<T, 64>(D, inv, lse_s, out_s, out, lse, st)
-                : launch_merge<T, 128>(D, inv, lse_s, out_s, out, lse, st);
+  s = D.d == 64 ? launch_merge<T, 64>(D, inv, lse, out_r, out, st)
+                : launch_merge<T, 128>(D, inv, lse, out_r, out, st);
   if (s != LSH_OK) return s;
   return mark(ev, 8, st);
 }
