@@ -162,7 +162,7 @@ lsh_status lsh_attn_get_diag(const void *workspace, void *stream, lsh_attn_diag 
  * every GPU that loads the library until the process exits.
  *   - buckets [B][H][Rn][n] int32 in; perm [B][H][Rn][n] int32 out (device).
  *   - A problem needs 256 + 4*B*H*Rn*nb*ceil(n / T) (rounded up to 256) +
- *     4*B*H*Rn*n bytes of scratch, T = 256 * clamp(16384 / nb, 1, 16); larger
+ *     4*B*H*Rn*n bytes of scratch, T = 256 * clamp(8192 / nb, 1, 8); larger
  *     problems return LSH_ERR_UNSUPPORTED and write nothing (use lsh_attn_sort).
  *   - The first call on a device looks up the scratch's device address (with
  *     that device current) and caches it; make that first call before any

@@ -19,10 +19,11 @@ namespace lsh {
 
 constexpr int kSortSub = 256;  // tokens per warp sub-range
 
-// Warps per tile: per-warp counters take warps * nb * 4 bytes of shared memory.
+// Warps per tile: per-warp counters take warps * nb * 4 bytes of shared memory
+// (at most 32 KB, so two gathering CTAs share an SM).
 __host__ __device__ inline int sort_warps(int nb) {
-  int w = 16384 / nb;
-  return w < 1 ? 1 : (w > 16 ? 16 : w);
+  int w = 8192 / nb;
+  return w < 1 ? 1 : (w > 8 ? 8 : w);
 }
 __host__ __device__ inline int sort_tile(int nb) { return sort_warps(nb) * kSortSub; }
 

@@ -1,14 +1,16 @@
 // Stable counting sort fused with the gather of x and v rows into sorted
 // order, the rows streamed by TMA ("Reformer summary" (ttnews.xyz),
-// §局部敏感哈希注意力: order the tokens by bucket, then by position).
+// §局部敏感哈希注意力: order the tokens by bucket, then by position). Two CTAs
+// share an SM, so one's ranking overlaps the other's copying.
 //
 // Same ranks as k_sort_scatter (per-warp counts, scan over warps seeded by
 // the tile's offsets, stable ranks from __match_any_sync); the slots of the
 // whole tile go to shared memory first. The tile's rows are contiguous in x
-// and v (position order), so a TMA ring (3 stages of 32 KB, issued before
+// and v (position order), so a TMA ring (2 stages of 32 KB, issued before
 // the ranks are computed) streams them into shared memory, and the warps
 // copy each row to its slot with row-coalesced 16-byte stores, summing the
-// squares of x on the way for 1/||x||.
+// squares of x on the way for 1/||x||. Each warp's 256 bucket ids are loaded
+// once, up front, for both ranking passes.
 #pragma once
 
 #include "common.cuh"
@@ -17,7 +19,7 @@
 
 namespace lsh {
 
-constexpr int kGatherStages = 3;
+constexpr int kGatherStages = 2;
 constexpr int kGatherStageBytes = 32768;  // x and v rows of one chunk
 
 struct SortGatherPlan {
@@ -42,7 +44,7 @@ inline SortGatherPlan sort_gather_plan(int nb, int d, int esize) {
 // perm, inv, invnorm [seg][n]; xs, vs [seg][n][d]. tmx / tmv: x, v as
 // [BH * n][d] with boxes of chunk_rows x d, no swizzle.
 template <typename T>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(256, 2)
     k_sort_gather_tma(const __grid_constant__ CUtensorMap tmx,
                       const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ buckets,
                       const int32_t* __restrict__ hist, int32_t* __restrict__ perm,
@@ -95,9 +97,16 @@ __global__ void __launch_bounds__(512, 1)
   const int wend = min(n, wstart + kSortSub);
   const int32_t* bk = buckets + (int64_t)seg * n;
   int32_t* mybase = base + warp * nb;
-  for (int s0 = wstart; s0 < wend; s0 += 32) {
-    const int t = s0 + lane;
-    const int b = t < wend ? clamp_bucket(bk[t], nb) : -1;
+  constexpr int kSteps = kSortSub / 32;
+  int bks[kSteps];  // this warp's bucket ids, -1 past the end
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) {
+    const int t = wstart + 32 * i + lane;
+    bks[i] = t < wend ? clamp_bucket(bk[t], nb) : -1;
+  }
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) {
+    const int b = bks[i];
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
     if (b >= 0 && lane == __ffs(peers) - 1) mybase[b] += __popc(peers);
     __syncwarp();
@@ -114,9 +123,10 @@ __global__ void __launch_bounds__(512, 1)
   }
   __syncthreads();
   const int64_t so = (int64_t)seg * n;
-  for (int s0 = wstart; s0 < wend; s0 += 32) {
-    const int t = s0 + lane;
-    const int b = t < wend ? clamp_bucket(bk[t], nb) : -1;
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) {
+    const int t = wstart + 32 * i + lane;
+    const int b = bks[i];
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
     int slot = 0;
     if (b >= 0) slot = mybase[b] + __popc(peers & lanemask_lt());
