@@ -50,21 +50,21 @@ STAGE_KERNEL = {"hash": "hash_mma", "sort_gather": "sort_scatter_gather",
 # of the file at capture time); see profiles/.
 NCU_TRAFFIC = {
     "hash_prep": {"bytes": 532000, "file": "hash_tc.cuh",
-        "sha256": "fd7b1da74b7ccb46fa154ea28d82c754ea1ba45bfdd1c9d9882f40c3c4fe2ea7"},
-    "hash_mma": {"bytes": 146183000, "file": "hash_tc.cuh",
-        "sha256": "fd7b1da74b7ccb46fa154ea28d82c754ea1ba45bfdd1c9d9882f40c3c4fe2ea7"},
-    "hash_refine": {"bytes": 2043999, "file": "hash_tc.cuh",
-        "sha256": "fd7b1da74b7ccb46fa154ea28d82c754ea1ba45bfdd1c9d9882f40c3c4fe2ea7"},
+        "sha256": "2b59d93de7b38217746a2913d0c68d626e2c4b7bc56d86102676880387173286"},
+    "hash_mma": {"bytes": 145883000, "file": "hash_tc.cuh",
+        "sha256": "2b59d93de7b38217746a2913d0c68d626e2c4b7bc56d86102676880387173286"},
+    "hash_refine": {"bytes": 2050000, "file": "hash_tc.cuh",
+        "sha256": "2b59d93de7b38217746a2913d0c68d626e2c4b7bc56d86102676880387173286"},
     "sort_hist": {"bytes": 8393000, "file": "sort.cuh",
-        "sha256": "78dde6d10c34979fa002a0f5e893d594535ca454bedca2ed29195ad246d2ef5a"},
-    "sort_scan": {"bytes": 2102000, "file": "sort.cuh",
-        "sha256": "78dde6d10c34979fa002a0f5e893d594535ca454bedca2ed29195ad246d2ef5a"},
-    "sort_scatter_gather": {"bytes": 1423398000, "file": "sort.cuh",
-        "sha256": "78dde6d10c34979fa002a0f5e893d594535ca454bedca2ed29195ad246d2ef5a"},
-    "chunk_attention": {"bytes": 2127058000, "file": "attn_tc.cuh",
-        "sha256": "a7fb05db1c0966392c14da11f5d33b9c4854904f9509f21acdacc187a3522449"},
-    "unsort_merge": {"bytes": 1227627000, "file": "merge.cuh",
-        "sha256": "b0c7ab1f33ff564b578073c8d8eb0b5bee9357cc6c2f8c04e8c21868a6947540"},
+        "sha256": "bb18c7ce75121f48157bba07d459db2fb295f4bb5d321eeaf0abcc010ec71cb7"},
+    "sort_scan": {"bytes": 4199000, "file": "sort.cuh",
+        "sha256": "bb18c7ce75121f48157bba07d459db2fb295f4bb5d321eeaf0abcc010ec71cb7"},
+    "sort_scatter_gather": {"bytes": 1411537000, "file": "sort_tma.cuh",
+        "sha256": "5f1e2222ff32e16d9196fd996834ecd1cfd0ed703df3ba11f6338726720cdce7"},
+    "chunk_attention": {"bytes": 2193920000, "file": "attn_tc.cuh",
+        "sha256": "6ea4d13c9febd5a1482d522a79666e3b01a39e11cc3c58cd4634353d75c7d54f"},
+    "unsort_merge": {"bytes": 1218285000, "file": "merge.cuh",
+        "sha256": "268533ed7ffa49aca75930c1f680445ee95797791f930f35f6b02c08748d885f"},
 }
 
 

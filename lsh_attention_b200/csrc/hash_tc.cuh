@@ -145,26 +145,47 @@ __global__ void __launch_bounds__(128)
       bv[e] = -INFINITY;
       bi[e] = 0x7fffffff;
     }
-    for (int j = tid; j < half; j += 128) {
-      const uint4* rr = reinterpret_cast<const uint4*>(Rr + (int64_t)j * D);
-      double acc[E];
+    // register tile: C columns x E tokens per thread; every column's sum still
+    // runs over k = 0..d-1 in order
+    constexpr int C = 4;
+    for (int j0 = tid; j0 < half; j0 += 128 * C) {
+      double acc[C][E];
+      const uint4* rr[C];
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = 0.0;
-#pragma unroll 2
-      for (int c = 0; c < D / 8; ++c) {
-        float f[8];
-        Vec16<__nv_bfloat16>::unpack(__ldg(rr + c), f);
+      for (int c = 0; c < C; ++c) {
+        const int j = min(j0 + 128 * c, half - 1);
+        rr[c] = reinterpret_cast<const uint4*>(Rr + (int64_t)j * D);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[c][e] = 0.0;
+      }
+#pragma unroll 1
+      for (int k8 = 0; k8 < D / 8; ++k8) {
+        float f[C][8];
+#pragma unroll
+        for (int c = 0; c < C; ++c) Vec16<__nv_bfloat16>::unpack(__ldg(rr[c] + k8), f[c]);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const double rv = (double)f[u];
+          double xv[E];
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[e] = fma(xs[e][c * 8 + u], rv, acc[e]);
+          for (int e = 0; e < E; ++e) xv[e] = xs[e][k8 * 8 + u];
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            const double rv = (double)f[c][u];
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[c][e] = fma(xv[e], rv, acc[c][e]);
+          }
         }
       }
 #pragma unroll
-      for (int e = 0; e < E; ++e) {
-        argmax_update(acc[e], j, bv[e], bi[e]);
-        argmax_update(-acc[e], half + j, bv[e], bi[e]);
+      for (int c = 0; c < C; ++c) {
+        const int j = j0 + 128 * c;
+        if (j < half) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            argmax_update(acc[c][e], j, bv[e], bi[e]);
+            argmax_update(-acc[c][e], half + j, bv[e], bi[e]);
+          }
+        }
       }
     }
 #pragma unroll
