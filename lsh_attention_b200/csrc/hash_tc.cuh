@@ -225,38 +225,81 @@ struct HashTcArgs {
 };
 
 // Running top-2 of |p| with the argmax and its signed value.
-struct Top2 {
-  float m1, m2, sv;
-  int idx;
+// Top-two tracker of |p_j| over one token's columns, fed 16 columns at a
+// time. Per batch it takes the batch maximum (a tree of 15 max operations)
+// and keeps the whole batch only when that maximum leads; the argmax, its
+// sign and the largest value beside it are found once, in the lead batch,
+// when the round is done. The second largest |p| overall is the larger of
+// that in-batch value and the largest maximum of the other batches, so the
+// result equals a column-by-column top-two scan, at about two operations per
+// value instead of six.
+struct BatchLead {
+  float m1;     // largest |p| so far (-1 before the first batch)
+  float m2o;    // largest batch maximum outside the lead batch
+  float s[16];  // the lead batch's signed values
+  int j0;       // its first column
   __device__ __forceinline__ void reset() {
-    m1 = 0.f;
-    m2 = 0.f;
-    sv = 0.f;
-    idx = 0;
+    m1 = -1.f;
+    m2o = 0.f;
+    j0 = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) s[k] = 0.f;
   }
-  __device__ __forceinline__ void add(float v, int j) {
-    const float a = fabsf(v);
-    const bool gt = a > m1;
-    m2 = gt ? m1 : fmaxf(m2, a);
-    idx = gt ? j : idx;
-    sv = gt ? v : sv;
-    m1 = gt ? a : m1;
+  __device__ __forceinline__ void add(const float (&w)[16], int jb) {
+    float t[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t[k] = fmaxf(fabsf(w[2 * k]), fabsf(w[2 * k + 1]));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) t[k] = fmaxf(t[k], t[k + 4]);
+    const float bm = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3]));
+    const bool gt = bm > m1;  // the earlier batch keeps the lead on a tie
+    m2o = gt ? fmaxf(m2o, m1) : fmaxf(m2o, bm);
+    m1 = gt ? bm : m1;
+    j0 = gt ? jb : j0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) s[k] = gt ? w[k] : s[k];
   }
-  // Fold another tracker in: the larger first value wins (lower index on a
-  // tie); the second value is the largest of the rest.
-  __device__ __forceinline__ void merge(float om1, float om2, int oidx, float osv) {
-    if (om1 > m1 || (om1 == m1 && oidx < idx)) {
-      m2 = fmaxf(fmaxf(om2, m2), m1);
-      m1 = om1;
-      idx = oidx;
-      sv = osv;
+  // Largest |p|, second largest, argmax column and its signed value; all
+  // zero when no batch was added.
+  __device__ __forceinline__ void finish(float& om1, float& om2, int& oidx, float& osv) const {
+    float a1 = -1.f, a2 = 0.f, sv = 0.f;
+    int k1 = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float a = fabsf(s[k]);
+      const bool gt = a > a1;  // lowest column on a tie
+      a2 = gt ? fmaxf(a2, a1) : fmaxf(a2, a);
+      k1 = gt ? k : k1;
+      sv = gt ? s[k] : sv;
+      a1 = gt ? a : a1;
+    }
+    if (m1 < 0.f) {
+      om1 = 0.f;
+      om2 = 0.f;
+      oidx = 0;
+      osv = 0.f;
     } else {
-      m2 = fmaxf(fmaxf(om2, m2), om1);
+      om1 = a1;
+      om2 = fmaxf(a2, m2o);
+      oidx = j0 + k1;
+      osv = sv;
     }
   }
 };
 
-constexpr int kHashLanesIlp = 4;  // independent trackers per thread (ILP)
+// Merge rule for the per-warp results of one token: the larger first value
+// wins (lower column on a tie); the second value is the largest of the rest.
+__device__ __forceinline__ void top2_merge(float& m1, float& m2, int& idx, float& sv, float om1,
+                                           float om2, int oidx, float osv) {
+  if (om1 > m1 || (om1 == m1 && oidx < idx)) {
+    m2 = fmaxf(fmaxf(om2, m2), m1);
+    m1 = om1;
+    idx = oidx;
+    sv = osv;
+  } else {
+    m2 = fmaxf(fmaxf(om2, m2), om1);
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kHashWarps * 32, 1)
@@ -411,9 +454,8 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
       }
       bool stop = false;
       for (int rl = 0; rl < gr; ++rl, ++rc) {
-        Top2 st[kHashLanesIlp];
-#pragma unroll
-        for (int i = 0; i < kHashLanesIlp; ++i) st[i].reset();
+        BatchLead st;
+        st.reset();
         for (int c = 0; ok && c < p.ch; ++c, ++u) {
           const int ab = u & 1, uk = u >> 1;
           if (!mbar_wait(acc_full + ab, uk & 1)) {
@@ -423,43 +465,58 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
           }
           tc_fence_after();
           const uint32_t tbase = tmem + tlane + ab * p.tmem_cols;
-          // this warp's 16-column batches are h, h + 3, ...: two loads in
-          // flight per wait
+          // This warp's 16-column batches are h, h + 3, h + 6, ... (K of
+          // them). Three register buffers rotate so that two loads are in
+          // flight while two batches are reduced; one wait per two batches.
           constexpr int P = kHashEpiPerQuad;
-          for (int i0 = 0; P * i0 + h < nbatch; i0 += 2) {
-            uint32_t v[2][16];
+          const int K = (nbatch - h + P - 1) / P;
+          auto ld = [&](uint32_t(&v)[16], int i) {
+            if (i < K) tmem_ld16(tbase + (h + P * i) * 16, v);
+          };
+          auto take = [&](const uint32_t(&v)[16], int i) {
+            if (i >= K) return;
+            const int j0 = c * p.nc + (h + P * i) * 16;
+            float w[16];
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
-              if (h + P * (i0 + i) < nbatch) tmem_ld16(tbase + (h + P * (i0 + i)) * 16, v[i]);
-            tmem_wait_ld();
+            for (int k = 0; k < 16; ++k) w[k] = __uint_as_float(v[k]);
+            if (j0 + 16 > p.half) {  // columns past b/2 are padding: |p| = 0
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const int b = h + P * (i0 + i);
-              if (b < nbatch) {
-                const int j0 = c * p.nc + b * 16;
-                if (j0 + 16 <= p.half) {
-#pragma unroll
-                  for (int k = 0; k < 16; ++k)
-                    st[k % kHashLanesIlp].add(__uint_as_float(v[i][k]), j0 + k);
-                } else {
-#pragma unroll
-                  for (int k = 0; k < 16; ++k)
-                    if (j0 + k < p.half)
-                      st[k % kHashLanesIlp].add(__uint_as_float(v[i][k]), j0 + k);
-                }
-              }
+              for (int k = 0; k < 16; ++k)
+                if (j0 + k >= p.half) w[k] = 0.f;
             }
+            st.add(w, j0);
+          };
+          uint32_t A[16], B[16], C[16];
+          ld(A, 0);
+          ld(B, 1);
+          tmem_wait_ld_regs(A, B);
+          for (int i = 0; i < K; i += 6) {
+            ld(C, i + 2);
+            take(A, i);
+            ld(A, i + 3);
+            take(B, i + 1);
+            tmem_wait_ld_regs(C, A);
+            ld(B, i + 4);
+            take(C, i + 2);
+            ld(C, i + 5);
+            take(A, i + 3);
+            tmem_wait_ld_regs(B, C);
+            ld(A, i + 6);
+            take(B, i + 4);
+            ld(B, i + 7);
+            take(C, i + 5);
+            tmem_wait_ld_regs(A, B);
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(acc_empty + ab);  // accumulator free for the next MMA
         }
-#pragma unroll
-        for (int i = 1; i < kHashLanesIlp; ++i) st[0].merge(st[i].m1, st[i].m2, st[i].idx, st[i].sv);
+        float m1, m2, sv;
+        int idx;
+        st.finish(m1, m2, idx, sv);
         // combine the warps of this quadrant, then decide
         float4* slot = comb + (((rc & 1) * 4 + q) * (kHashEpiPerQuad - 1)) * 32 + lane;
-        if (h > 0)
-          slot[(h - 1) * 32] = make_float4(st[0].m1, st[0].m2, __int_as_float(st[0].idx), st[0].sv);
+        if (h > 0) slot[(h - 1) * 32] = make_float4(m1, m2, __int_as_float(idx), sv);
         asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kHashEpiPerQuad) : "memory");
         stop = *abort_flag != 0;
         if (stop) break;
@@ -467,10 +524,8 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
 #pragma unroll
           for (int o_ = 0; o_ < kHashEpiPerQuad - 1; ++o_) {
             const float4 o = slot[o_ * 32];
-            st[0].merge(o.x, o.y, __float_as_int(o.z), o.w);
+            top2_merge(m1, m2, idx, sv, o.x, o.y, __float_as_int(o.z), o.w);
           }
-          const float m1 = st[0].m1, m2 = st[0].m2, sv = st[0].sv;
-          const int idx = st[0].idx;
           if (t < a.n) {
             const int r = r0 + rl;
             const float tau = kTieFactor * (float)D * 1.1920929e-7f * xnorm * rnorm[r];
