@@ -7,13 +7,15 @@
 //   * the rotations of a group of rounds stay resident in shared memory
 //     (transposed to K-major by k_hash_prep, loaded once by TMA);
 //   * warp 0 streams 128-token tiles of x with TMA (double-buffered);
-//   * warp 1 issues tcgen05.mma (M = 128 tokens, N <= 256 columns, K = d)
+//   * warp 1 issues tcgen05.mma (M = 128 tokens, N <= 192 columns, K = d)
 //     into one of two TMEM accumulators, so the next unit's MMA overlaps the
 //     epilogue of the current one;
 //   * warps 2..13 read the fp32 projections with tcgen05.ld and keep, per
 //     token, the largest and second largest |p_j|, the argmax and its sign
-//     (three warps per TMEM lane quadrant, each on every third 16-column
-//     batch).
+//     (three warps per TMEM lane quadrant, each on a contiguous range of at
+//     most four 16-column batches, all loaded before one wait). The
+//     accumulator is handed back to the MMA as soon as a warp's loads are
+//     done, and ||x|| is summed by the warps that do not decide.
 // Exactness: the fp32 accumulation of d bf16 products is within
 // d * 2^-23 * sum_k |x_k R_kj| <= d * 2^-23 * ||x|| ||R_j|| of the exact sum,
 // whatever the order or rounding of the additions. When the top two |p| are
@@ -29,8 +31,9 @@
 namespace lsh {
 
 constexpr int kHashTile = 128;       // tokens per tile (MMA M)
-constexpr int kHashMaxN = 256;       // columns per MMA (N)
 constexpr int kHashEpiPerQuad = 3;   // epilogue warps per TMEM lane quadrant
+constexpr int kHashMaxBatches = 4;   // 16-column batches per epilogue warp and unit
+constexpr int kHashMaxN = 16 * kHashMaxBatches * kHashEpiPerQuad;  // columns per MMA (N): 192
 constexpr int kHashWarps = 2 + 4 * kHashEpiPerQuad;  // 0: TMA, 1: MMA, rest: epilogue
 constexpr float kTieFactor = 4.0f;   // margin threshold / accumulation error bound
 constexpr int kHashSmemBudget = 227 * 1024;
@@ -225,39 +228,51 @@ struct HashTcArgs {
 };
 
 // Running top-2 of |p| with the argmax and its signed value.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Top-two tracker of |p_j| over one token's columns, fed 16 columns at a
-// time. Per batch it takes the batch maximum (a tree of 15 max operations)
-// and keeps the whole batch only when that maximum leads; the argmax, its
-// sign and the largest value beside it are found once, in the lead batch,
-// when the round is done. The second largest |p| overall is the larger of
-// that in-batch value and the largest maximum of the other batches, so the
-// result equals a column-by-column top-two scan, at about two operations per
-// value instead of six.
+// time. Per batch it takes the batch maximum (a tree of three-input max
+// operations) and keeps the whole batch only when that maximum leads; the
+// argmax, its sign and the largest value beside it are found once, in the
+// lead batch, when the round is done. The second largest |p| overall is the
+// larger of that in-batch value and the largest maximum of the other
+// batches, so the result equals a column-by-column top-two scan. Columns
+// past b/2 (zero rows of the padded rotation) give p = 0 exactly and never
+// lead: the first of equal maxima keeps the lead, and a zero maximum is a
+// tie that is re-decided.
 struct BatchLead {
   float m1;     // largest |p| so far (-1 before the first batch)
   float m2o;    // largest batch maximum outside the lead batch
+  float j0;     // first column of the lead batch (exact in fp32)
   float s[16];  // the lead batch's signed values
-  int j0;       // its first column
   __device__ __forceinline__ void reset() {
     m1 = -1.f;
     m2o = 0.f;
-    j0 = 0;
+    j0 = 0.f;
 #pragma unroll
     for (int k = 0; k < 16; ++k) s[k] = 0.f;
   }
-  __device__ __forceinline__ void add(const float (&w)[16], int jb) {
-    float t[8];
+  // Batch of 16 values starting at column jb.
+  __device__ __forceinline__ void add(const uint32_t (&v)[16], float jb) {
+    float w[16];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) t[k] = fmaxf(fabsf(w[2 * k]), fabsf(w[2 * k + 1]));
+    for (int k = 0; k < 16; ++k) w[k] = __uint_as_float(v[k]);
+    const float u0 = fmax3(fabsf(w[0]), fabsf(w[1]), fabsf(w[2]));
+    const float u1 = fmax3(fabsf(w[3]), fabsf(w[4]), fabsf(w[5]));
+    const float u2 = fmax3(fabsf(w[6]), fabsf(w[7]), fabsf(w[8]));
+    const float u3 = fmax3(fabsf(w[9]), fabsf(w[10]), fabsf(w[11]));
+    const float u4 = fmax3(fabsf(w[12]), fabsf(w[13]), fabsf(w[14]));
+    const float bm = fmaxf(fmax3(u0, u1, u2), fmax3(u3, u4, fabsf(w[15])));
+    const bool lead = bm > m1;        // the earlier batch keeps the lead on a tie
+    m2o = fmaxf(m2o, fminf(bm, m1));  // the batch that does not lead
+    m1 = fmaxf(m1, bm);
+    j0 = lead ? jb : j0;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) t[k] = fmaxf(t[k], t[k + 4]);
-    const float bm = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3]));
-    const bool gt = bm > m1;  // the earlier batch keeps the lead on a tie
-    m2o = gt ? fmaxf(m2o, m1) : fmaxf(m2o, bm);
-    m1 = gt ? bm : m1;
-    j0 = gt ? jb : j0;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) s[k] = gt ? w[k] : s[k];
+    for (int k = 0; k < 16; ++k) s[k] = lead ? w[k] : s[k];
   }
   // Largest |p|, second largest, argmax column and its signed value; all
   // zero when no batch was added.
@@ -281,7 +296,7 @@ struct BatchLead {
     } else {
       om1 = a1;
       om2 = fmaxf(a2, m2o);
-      oidx = j0 + k1;
+      oidx = (int)j0 + k1;
       osv = sv;
     }
   }
@@ -321,7 +336,10 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
   uint64_t* acc_empty = bars + 7;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
-  float4* comb = reinterpret_cast<float4*>(bars + 16);  // [2][4][2][32]
+  constexpr int PO = kHashEpiPerQuad - 1;  // warps of a quadrant that report to h = 0
+  float4* comb = reinterpret_cast<float4*>(bars + 16);  // [2][4][PO][32]
+  float* ssb = reinterpret_cast<float*>(comb + 2 * 4 * PO * 32);  // [2][4][PO][32]
+  float* rn_s = ssb + 2 * 4 * PO * 32;                             // [rounds <= 16]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x / a.ctas_per_group;
@@ -333,13 +351,15 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
     mbar_init(r_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(x_full + i, 1);
-      mbar_init(x_empty + i, 1 + 4);  // MMA commit + 4 norm-reading warps
+      mbar_init(x_empty + i, 1 + 4 * PO);  // MMA commit + the norm-reading warps
       mbar_init(acc_full + i, 1);
       mbar_init(acc_empty + i, 4 * kHashEpiPerQuad);  // every epilogue warp
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (threadIdx.x < a.rounds)  // per-round bound of max_j ||R_j|| (k_hash_prep)
+    rn_s[threadIdx.x] = reinterpret_cast<const float*>(a.hdr->pad)[threadIdx.x];
   if (warp == 1) tmem_alloc(tmem_slot, 2 * p.tmem_cols);
   tc_fence_before();
   __syncthreads();
@@ -378,7 +398,20 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kHashTile, p.nc);
+      // Descriptors of the first K-step of each operand; K-step kk adds a
+      // fixed offset, in 16-byte units, to the start-address field in the low
+      // word (shared addresses stay below 256 KB, so the field never carries).
+      const uint64_t xd0 = desc_kmajor_sw128(smem_u32(xbuf));
+      const uint64_t xd1 = desc_kmajor_sw128(smem_u32(xbuf + KH * XBOX));
+      const uint64_t rd0 = desc_kmajor_sw128(smem_u32(rbuf));
+      const uint32_t desc_hi = (uint32_t)(xd0 >> 32);  // same for every operand
+      const uint32_t r_chunk = (uint32_t)(KH * p.nc * 128) >> 4;
+      const uint32_t r_half = (uint32_t)(p.nc * 128) >> 4;  // next 64 columns of K
+      // the last chunk of a round stops at the first multiple of 16 columns
+      // past b/2
+      const uint32_t idesc_full = idesc_bf16_f32(kHashTile, p.nc);
+      const uint32_t idesc_last =
+          idesc_bf16_f32(kHashTile, min(p.nc, (p.half - (p.ch - 1) * p.nc + 15) & ~15));
       bool ok = mbar_wait(r_full, 0);
       if (!ok) fail();
       int it = 0, u = 0;
@@ -386,21 +419,23 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
         const int xb = it & 1, xk = it >> 1;
         if (!mbar_wait(x_full + xb, xk & 1)) { fail(); break; }
         tc_fence_after();
-        const uint32_t xaddr = smem_u32(xbuf + xb * KH * XBOX);
+        const uint32_t a_lo = (uint32_t)(xb ? xd1 : xd0);
         for (int rl = 0; rl < gr && ok; ++rl) {
           for (int c = 0; c < p.ch; ++c, ++u) {
             const int ab = u & 1, uk = u >> 1;
             if (uk > 0 && !mbar_wait(acc_empty + ab, (uk - 1) & 1)) { fail(); ok = false; break; }
             if (*abort_flag) { ok = false; break; }
             tc_fence_after();
-            const uint32_t raddr =
-                smem_u32(rbuf + (size_t)(rl * p.ch + c) * KH * p.nc * 128);
+            const uint32_t b_lo = (uint32_t)rd0 + (uint32_t)(rl * p.ch + c) * r_chunk;
             const uint32_t d_tmem = tmem + ab * p.tmem_cols;
+            const uint32_t idesc = c == p.ch - 1 ? idesc_last : idesc_full;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const int kh = kk >> 2, ks = kk & 3;
-              const uint64_t adesc = desc_kmajor_sw128(xaddr + kh * XBOX + ks * 32);
-              const uint64_t bdesc = desc_kmajor_sw128(raddr + kh * p.nc * 128 + ks * 32);
+              const uint64_t adesc =
+                  ((uint64_t)desc_hi << 32) | (a_lo + (uint32_t)((kh * XBOX + ks * 32) >> 4));
+              const uint64_t bdesc =
+                  ((uint64_t)desc_hi << 32) | (b_lo + kh * r_half + (uint32_t)(ks * 2));
               mma_bf16_ss(d_tmem, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
             }
             mma_commit(acc_full + ab);
@@ -413,11 +448,9 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
     // ------------------------------------------------------------ epilogue
     const int e = warp - 2;
     const int q = warp & 3;       // TMEM lane quadrant this warp may access
-    const int h = e >> 2;         // this warp takes the 16-column batches b = h (mod 3)
+    const int h = e >> 2;         // rank of this warp in its quadrant
     const int row = q * 32 + lane;
     const uint32_t tlane = (uint32_t)(q * 32) << 16;
-    const float* rnorm = reinterpret_cast<const float*>(a.hdr->pad);
-    const int nbatch = p.nc / 16;
     int it = 0, u = 0, rc = 0;
     for (int tile = li; tile < a.tiles; tile += a.ctas_per_group, ++it) {
       const int xb = it & 1, xk = it >> 1;
@@ -426,28 +459,25 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
       // Failures set abort_flag before the next named barrier, so both warps
       // of a quadrant leave the loop after the same barrier.
       bool ok = true;
-      float xnorm = 0.f;
-      if (h == 0) {
+      // ||x_row||^2 in parts: warp h >= 1 sums the row's 16-byte chunks
+      // cc = h - 1 (mod PO) from the swizzled tile (chunk c of a 128-byte
+      // line sits at slot c ^ (row % 8)). Warp h = 0, which decides, reads
+      // the partial sums at each round's combine.
+      float ss = 0.f;
+      if (h > 0) {
         if (!mbar_wait(x_full + xb, xk & 1)) {
           fail();
           ok = false;
         } else {
-          // ||x_row|| from the swizzled tile: 16-byte chunk c of a row sits at
-          // slot c ^ (row % 8) of its 128-byte line.
-          float ss = 0.f;
+#pragma unroll 2
+          for (int cc = h - 1; cc < KH * 8; cc += PO) {
+            const unsigned char* line = xbuf + (xb * KH + (cc >> 3)) * XBOX + row * 128;
+            const uint4 v = *reinterpret_cast<const uint4*>(line + (((cc & 7) ^ (row & 7)) << 4));
+            float f[8];
+            Vec16<__nv_bfloat16>::unpack(v, f);
 #pragma unroll
-          for (int kh = 0; kh < KH; ++kh) {
-            const unsigned char* line = xbuf + (xb * KH + kh) * XBOX + row * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const uint4 v = *reinterpret_cast<const uint4*>(line + ((c ^ (row & 7)) << 4));
-              float f[8];
-              Vec16<__nv_bfloat16>::unpack(v, f);
-#pragma unroll
-              for (int k = 0; k < 8; ++k) ss = fmaf(f[k], f[k], ss);
-            }
+            for (int k = 0; k < 8; ++k) ss = fmaf(f[k], f[k], ss);
           }
-          xnorm = sqrtf(ss) * 1.0001f;  // covers the fp32 rounding of the norm
           __syncwarp();
           if (lane == 0) mbar_arrive(x_empty + xb);
         }
@@ -465,70 +495,56 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
           }
           tc_fence_after();
           const uint32_t tbase = tmem + tlane + ab * p.tmem_cols;
-          // This warp's 16-column batches are h, h + 3, h + 6, ... (K of
-          // them). Three register buffers rotate so that two loads are in
-          // flight while two batches are reduced; one wait per two batches.
-          constexpr int P = kHashEpiPerQuad;
-          const int K = (nbatch - h + P - 1) / P;
-          auto ld = [&](uint32_t(&v)[16], int i) {
-            if (i < K) tmem_ld16(tbase + (h + P * i) * 16, v);
-          };
-          auto take = [&](const uint32_t(&v)[16], int i) {
-            if (i >= K) return;
-            const int j0 = c * p.nc + (h + P * i) * 16;
-            float w[16];
+          // The chunk's batches are split over the quadrant's warps, at
+          // most kHashMaxBatches each, the larger shares to the higher ranks
+          // (h = 0 also decides). A warp's loads are issued together and
+          // waited for once: one TMEM round trip per unit.
+          const int nbc = (min(p.nc, p.half - c * p.nc) + 15) >> 4;
+          const int base = nbc / kHashEpiPerQuad, extra_from = kHashEpiPerQuad - nbc % kHashEpiPerQuad;
+          const int K = base + (h >= extra_from ? 1 : 0);
+          const int b_lo = h * base + max(0, h - extra_from);
+          uint32_t V[kHashMaxBatches][16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) w[k] = __uint_as_float(v[k]);
-            if (j0 + 16 > p.half) {  // columns past b/2 are padding: |p| = 0
-#pragma unroll
-              for (int k = 0; k < 16; ++k)
-                if (j0 + k >= p.half) w[k] = 0.f;
-            }
-            st.add(w, j0);
-          };
-          uint32_t A[16], B[16], C[16];
-          ld(A, 0);
-          ld(B, 1);
-          tmem_wait_ld_regs(A, B);
-          for (int i = 0; i < K; i += 6) {
-            ld(C, i + 2);
-            take(A, i);
-            ld(A, i + 3);
-            take(B, i + 1);
-            tmem_wait_ld_regs(C, A);
-            ld(B, i + 4);
-            take(C, i + 2);
-            ld(C, i + 5);
-            take(A, i + 3);
-            tmem_wait_ld_regs(B, C);
-            ld(A, i + 6);
-            take(B, i + 4);
-            ld(B, i + 7);
-            take(C, i + 5);
-            tmem_wait_ld_regs(A, B);
-          }
+          for (int k = 0; k < kHashMaxBatches; ++k)
+            if (k < K) tmem_ld16(tbase + (b_lo + k) * 16, V[k]);
+          tmem_wait_ld_regs(V);
+          // the values are in registers: the accumulator is free for the MMA
+          // of the unit after next while they are reduced
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty + ab);  // accumulator free for the next MMA
+          if (lane == 0) mbar_arrive(acc_empty + ab);
+          const float jb0 = (float)(c * p.nc + b_lo * 16);
+#pragma unroll
+          for (int k = 0; k < kHashMaxBatches; ++k)
+            if (k < K) st.add(V[k], jb0 + 16.f * (float)k);
         }
         float m1, m2, sv;
         int idx;
         st.finish(m1, m2, idx, sv);
         // combine the warps of this quadrant, then decide
-        float4* slot = comb + (((rc & 1) * 4 + q) * (kHashEpiPerQuad - 1)) * 32 + lane;
-        if (h > 0) slot[(h - 1) * 32] = make_float4(m1, m2, __int_as_float(idx), sv);
+        float4* slot = comb + (((rc & 1) * 4 + q) * PO) * 32 + lane;
+        float* sslot = ssb + (((rc & 1) * 4 + q) * PO) * 32 + lane;
+        if (h > 0) {
+          slot[(h - 1) * 32] = make_float4(m1, m2, __int_as_float(idx), sv);
+          sslot[(h - 1) * 32] = ss;
+        }
         asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kHashEpiPerQuad) : "memory");
         stop = *abort_flag != 0;
         if (stop) break;
         if (h == 0) {
 #pragma unroll
-          for (int o_ = 0; o_ < kHashEpiPerQuad - 1; ++o_) {
+          for (int o_ = 0; o_ < PO; ++o_) {
             const float4 o = slot[o_ * 32];
             top2_merge(m1, m2, idx, sv, o.x, o.y, __float_as_int(o.z), o.w);
           }
           if (t < a.n) {
             const int r = r0 + rl;
-            const float tau = kTieFactor * (float)D * 1.1920929e-7f * xnorm * rnorm[r];
+            // ||x|| rounded up past the fp32 rounding of its square sum
+            float sst = 0.f;
+#pragma unroll
+            for (int o_ = 0; o_ < PO; ++o_) sst += sslot[o_ * 32];
+            const float xnorm = sqrtf(sst) * 1.0001f;
+            const float tau = kTieFactor * (float)D * 1.1920929e-7f * xnorm * rn_s[r];
             const int bucket = idx + (sv < 0.f ? p.half : 0);
             const int64_t at = ((int64_t)bh * a.rounds + r) * a.n + t;
             a.buckets[at] = bucket;

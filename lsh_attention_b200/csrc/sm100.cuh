@@ -164,14 +164,38 @@ __device__ __forceinline__ void tmem_wait_ld() {
 // The same wait, naming the destination registers of the loads it completes
 // as operands, so the compiler cannot move a read of them above the wait
 // (the load asm defines them at its issue, before the data has arrived).
-__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[16], uint32_t (&b)[16]) {
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[4][16]) {
   asm volatile(
       "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]),
-        "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]),
-        "+r"(a[14]), "+r"(a[15]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]),
-        "+r"(b[5]), "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]),
-        "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15])
+      : "+r"(a[0][0]), "+r"(a[0][1]), "+r"(a[0][2]), "+r"(a[0][3]), "+r"(a[0][4]),
+        "+r"(a[0][5]), "+r"(a[0][6]), "+r"(a[0][7]), "+r"(a[0][8]), "+r"(a[0][9]),
+        "+r"(a[0][10]), "+r"(a[0][11]), "+r"(a[0][12]), "+r"(a[0][13]), "+r"(a[0][14]),
+        "+r"(a[0][15]), "+r"(a[1][0]), "+r"(a[1][1]), "+r"(a[1][2]), "+r"(a[1][3]),
+        "+r"(a[1][4]), "+r"(a[1][5]), "+r"(a[1][6]), "+r"(a[1][7]), "+r"(a[1][8]),
+        "+r"(a[1][9]), "+r"(a[1][10]), "+r"(a[1][11]), "+r"(a[1][12]), "+r"(a[1][13]),
+        "+r"(a[1][14]), "+r"(a[1][15]), "+r"(a[2][0]), "+r"(a[2][1]), "+r"(a[2][2]),
+        "+r"(a[2][3]), "+r"(a[2][4]), "+r"(a[2][5]), "+r"(a[2][6]), "+r"(a[2][7]),
+        "+r"(a[2][8]), "+r"(a[2][9]), "+r"(a[2][10]), "+r"(a[2][11]), "+r"(a[2][12]),
+        "+r"(a[2][13]), "+r"(a[2][14]), "+r"(a[2][15]), "+r"(a[3][0]), "+r"(a[3][1]),
+        "+r"(a[3][2]), "+r"(a[3][3]), "+r"(a[3][4]), "+r"(a[3][5]), "+r"(a[3][6]),
+        "+r"(a[3][7]), "+r"(a[3][8]), "+r"(a[3][9]), "+r"(a[3][10]), "+r"(a[3][11]),
+        "+r"(a[3][12]), "+r"(a[3][13]), "+r"(a[3][14]), "+r"(a[3][15])
+      :
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[3][16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(a[0][0]), "+r"(a[0][1]), "+r"(a[0][2]), "+r"(a[0][3]), "+r"(a[0][4]),
+        "+r"(a[0][5]), "+r"(a[0][6]), "+r"(a[0][7]), "+r"(a[0][8]), "+r"(a[0][9]),
+        "+r"(a[0][10]), "+r"(a[0][11]), "+r"(a[0][12]), "+r"(a[0][13]), "+r"(a[0][14]),
+        "+r"(a[0][15]), "+r"(a[1][0]), "+r"(a[1][1]), "+r"(a[1][2]), "+r"(a[1][3]),
+        "+r"(a[1][4]), "+r"(a[1][5]), "+r"(a[1][6]), "+r"(a[1][7]), "+r"(a[1][8]),
+        "+r"(a[1][9]), "+r"(a[1][10]), "+r"(a[1][11]), "+r"(a[1][12]), "+r"(a[1][13]),
+        "+r"(a[1][14]), "+r"(a[1][15]), "+r"(a[2][0]), "+r"(a[2][1]), "+r"(a[2][2]),
+        "+r"(a[2][3]), "+r"(a[2][4]), "+r"(a[2][5]), "+r"(a[2][6]), "+r"(a[2][7]),
+        "+r"(a[2][8]), "+r"(a[2][9]), "+r"(a[2][10]), "+r"(a[2][11]), "+r"(a[2][12]),
+        "+r"(a[2][13]), "+r"(a[2][14]), "+r"(a[2][15])
       :
       : "memory");
 }
