@@ -50,21 +50,21 @@ STAGE_KERNEL = {"hash": "hash_mma", "sort_gather": "sort_scatter_gather",
 # of the file at capture time); see profiles/.
 NCU_TRAFFIC = {
     "hash_prep": {"bytes": 532000, "file": "hash_tc.cuh",
-        "sha256": "2b59d93de7b38217746a2913d0c68d626e2c4b7bc56d86102676880387173286"},
-    "hash_mma": {"bytes": 145883000, "file": "hash_tc.cuh",
-        "sha256": "2b59d93de7b38217746a2913d0c68d626e2c4b7bc56d86102676880387173286"},
+        "sha256": "684e370eca8f9f6eab6507cda92eff0e6f320859492c5b7d1d373eb0080708a5"},
+    "hash_mma": {"bytes": 144067000, "file": "hash_tc.cuh",
+        "sha256": "684e370eca8f9f6eab6507cda92eff0e6f320859492c5b7d1d373eb0080708a5"},
     "hash_refine": {"bytes": 2050000, "file": "hash_tc.cuh",
-        "sha256": "2b59d93de7b38217746a2913d0c68d626e2c4b7bc56d86102676880387173286"},
+        "sha256": "684e370eca8f9f6eab6507cda92eff0e6f320859492c5b7d1d373eb0080708a5"},
     "sort_hist": {"bytes": 8393000, "file": "sort.cuh",
         "sha256": "bb18c7ce75121f48157bba07d459db2fb295f4bb5d321eeaf0abcc010ec71cb7"},
     "sort_scan": {"bytes": 4199000, "file": "sort.cuh",
         "sha256": "bb18c7ce75121f48157bba07d459db2fb295f4bb5d321eeaf0abcc010ec71cb7"},
-    "sort_scatter_gather": {"bytes": 1411537000, "file": "sort_tma.cuh",
+    "sort_scatter_gather": {"bytes": 1409771000, "file": "sort_tma.cuh",
         "sha256": "5f1e2222ff32e16d9196fd996834ecd1cfd0ed703df3ba11f6338726720cdce7"},
-    "chunk_attention": {"bytes": 2193920000, "file": "attn_tc.cuh",
-        "sha256": "6ea4d13c9febd5a1482d522a79666e3b01a39e11cc3c58cd4634353d75c7d54f"},
-    "unsort_merge": {"bytes": 1218285000, "file": "merge.cuh",
-        "sha256": "268533ed7ffa49aca75930c1f680445ee95797791f930f35f6b02c08748d885f"},
+    "chunk_attention": {"bytes": 1654679000, "file": "attn_tc.cuh",
+        "sha256": "bad5498d5272605d7327ada9bc907ae21333a470122a2e0897b413a37963efad"},
+    "unsort_merge": {"bytes": 673733000, "file": "merge.cuh",
+        "sha256": "434e0ca452f2adcc23b4642755cd266872e0601d79c6d2c1704dabe29dfd4805"},
 }
 
 
@@ -91,9 +91,9 @@ def algorithmic(w: I.Workload) -> dict:
         "hash": {"bytes": X + Rn * w.d * (w.n_buckets // 2) * E + 4 * T * Rn,
                  "flops": 2 * T * w.d * (w.n_buckets // 2) * Rn},
         "sort_gather": {"bytes": 4 * T * Rn + 2 * X * Rn + 2 * X * Rn + 8 * T * Rn, "flops": 0},
-        "chunk_attention": {"bytes": 2 * X * Rn + 4 * T * Rn + T * Rn * w.d * 4 + 4 * T * Rn,
+        "chunk_attention": {"bytes": 2 * X * Rn + 4 * T * Rn + T * Rn * w.d * E + 4 * T * Rn,
                             "flops": 8 * m * w.d * T * Rn},
-        "unsort_merge": {"bytes": T * Rn * (4 * w.d + 8) + X, "flops": 0},
+        "unsort_merge": {"bytes": T * Rn * (E * w.d + 8) + X, "flops": 0},
     }
 
 

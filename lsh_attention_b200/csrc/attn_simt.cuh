@@ -10,7 +10,8 @@
 // The window is swept in blocks of 64 keys with a running max and sum, so
 // any chunk length up to 128 fits. This kernel serves fp32 inputs and chunk
 // lengths the tensor-core kernel does not take. Each round's output row is
-// written at the query's slot and its lse at the query's position.
+// written at the query's slot, in the input type, and its lse at the query's
+// position.
 #pragma once
 
 #include "common.cuh"
@@ -22,12 +23,12 @@ constexpr int kSimtKeys = 64;  // keys per block of the window sweep
 
 // grid (n / m, segments), block 256.
 // xs, vs [seg][n][d] sorted rows; perm, invnorm [seg][n];
-// out_r [seg][n][d] fp32 in slot order, lse [seg][n] fp32 in position order.
+// out_r [seg][n][d] in T, slot order; lse [seg][n] fp32 in position order.
 template <typename T, int D, int QPW>
 __global__ void __launch_bounds__(kSimtWarps * 32)
     k_attn_simt(const T* __restrict__ xs, const T* __restrict__ vs,
                 const int32_t* __restrict__ perm, const float* __restrict__ invnorm,
-                float* __restrict__ out_r, float* __restrict__ lse, int n, int m, int causal) {
+                T* __restrict__ out_r, float* __restrict__ lse, int n, int m, int causal) {
   constexpr int DP = D + 1;     // padded fp32 row: conflict-free per-lane key rows
   constexpr int DL = D / 32;    // output dims per lane
   extern __shared__ __align__(16) float sm[];
@@ -117,9 +118,9 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
     const int q = warp + i * kSimtWarps;
     if (q >= m) break;
     const float inv = 1.0f / lrun[i];
-    float* o = out_r + (so + q0 + q) * D;
+    T* o = out_r + (so + q0 + q) * D;
 #pragma unroll
-    for (int k = 0; k < DL; ++k) o[lane + 32 * k] = acc[i][k] * inv;
+    for (int k = 0; k < DL; ++k) o[lane + 32 * k] = Elem<T>::from_f(acc[i][k] * inv);
     if (lane == 0) lse[so + qpos[i]] = mrun[i] + logf(lrun[i]);
   }
 }

@@ -23,10 +23,13 @@
 //               dead S columns) as soon as it is computed; the row sum goes to
 //               the epilogue. A row whose only visible key is itself (the -1e5
 //               self logit) is flagged: its output is v of the query itself.
-//   warps 6..9  epilogue: O from TMEM, divided by the row sum, staged per warp
-//               in a 4 KB swizzled buffer (32 rows x 32 fp32) and written by
-//               TMA bulk stores (slot order), so every 128-byte line leaves the
-//               SM whole; the softmax writes lse at the query's position
+//   warps 6..9  epilogue: O from TMEM, divided by the row sum, rounded to
+//               bf16, staged per warp in a 4 KB swizzled buffer (32 rows x 64
+//               columns) and written by TMA bulk stores (slot order), so every
+//               128-byte line leaves the SM whole; the softmax writes lse at
+//               the query's position. Each round's output is kept in bf16: its
+//               rounding (relative 2^-9, before a convex combination over the
+//               rounds) is of the size of the final bf16 rounding of out.
 // TMEM: S[0] = [0, 192), S[1] = [192, 384), O = [384, 384 + d).
 #pragma once
 
@@ -47,7 +50,7 @@ struct AttnTcArgs {
   const float* invnorm;        // [S][n] 1/||x|| of the sorted rows (0 for a zero row)
   const int32_t* perm;         // [S][n] position of each slot
   const __nv_bfloat16* vs;     // [S][n][d] sorted v rows (self-only rows copy theirs)
-  float* out_r;                // [S][n][d] fp32, each round's output in slot order
+  __nv_bfloat16* out_r;        // [S][n][d] each round's output in slot order (TMA stores)
   float* lse;                  // [S][n] each round's lse by position (the caller's output)
   WsHeader* hdr;
   int n, causal, pairs_per_seg;
@@ -322,32 +325,31 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         const uint4* vr = reinterpret_cast<const uint4*>(a.vs + (seg * a.n + qs0 + lane) * (int64_t)D);
         unsigned char* stg = ostage + (warp - 6) * 32 * 128;
 #pragma unroll
-        for (int b = 0; b < D / 32; ++b) {
+        for (int b = 0; b < D / 64; ++b) {  // 64 columns (128 bytes of bf16) per store
           if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
           __syncwarp();
-          // row `lane`, 16-byte chunk c goes to slot c ^ (lane % 8) (128-byte swizzle)
+          // row `lane`, 16-byte chunk c (columns 64 b + 8 c ...) goes to slot
+          // c ^ (lane % 8) (128-byte swizzle)
           unsigned char* line = stg + lane * 128;
           if (inv > 0.f) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<float4*>(line + ((c ^ (lane & 7)) << 4)) = make_float4(
-                  __uint_as_float(o[b][4 * c]) * inv, __uint_as_float(o[b][4 * c + 1]) * inv,
-                  __uint_as_float(o[b][4 * c + 2]) * inv, __uint_as_float(o[b][4 * c + 3]) * inv);
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t* src = &o[2 * b + (c >> 2)][8 * (c & 3)];
+              *reinterpret_cast<uint4*>(line + ((c ^ (lane & 7)) << 4)) = make_uint4(
+                  pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv),
+                  pack_bf16x2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv),
+                  pack_bf16x2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv),
+                  pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv));
+            }
           } else {  // only the token itself is visible: its own value row
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              float f[8];
-              Vec16<__nv_bfloat16>::unpack(vr[b * 4 + c], f);
-              *reinterpret_cast<float4*>(line + (((2 * c) ^ (lane & 7)) << 4)) =
-                  make_float4(f[0], f[1], f[2], f[3]);
-              *reinterpret_cast<float4*>(line + (((2 * c + 1) ^ (lane & 7)) << 4)) =
-                  make_float4(f[4], f[5], f[6], f[7]);
-            }
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(line + ((c ^ (lane & 7)) << 4)) = vr[b * 8 + c];
           }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmo, stg, b * 32, (int)(seg * a.n) + qs0);
+            tma_store_2d(&tmo, stg, b * 64, (int)(seg * a.n) + qs0);
             bulk_commit();
           }
         }

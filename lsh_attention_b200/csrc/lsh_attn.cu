@@ -84,7 +84,7 @@ Layout layout_of(const Dims& D) {
   L.hist = take((size_t)D.S * D.nb * D.tiles * 4);
   L.xs = take(sn * D.d * D.esize);
   L.vs = take(sn * D.d * D.esize);
-  L.out_s = take(sn * D.d * 4);
+  L.out_s = take(sn * D.d * D.esize);  // each round's output rows, in the input type
   const HashTcPlan hp = hash_tc_plan(D.d, D.nb, D.rounds);
   L.rt = take((size_t)D.rounds * hp.ch * hp.nc * D.d * 2);  // R transposed (bf16 hash)
   L.refine = take(sn * 8);                             // near-tie queue of the bf16 hash
@@ -269,7 +269,7 @@ lsh_status launch_sort(const Dims& D, const int32_t* buckets, const void* x, con
 
 template <typename T, int DD, int QPW>
 lsh_status launch_attn_simt_q(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
-                              const float* invnorm, float* out_s, float* lse_s, cudaStream_t st) {
+                              const float* invnorm, T* out_s, float* lse_s, cudaStream_t st) {
   const size_t smem = attn_simt_smem(DD);
   auto kern = k_attn_simt<T, DD, QPW>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -283,7 +283,7 @@ lsh_status launch_attn_simt_q(const Dims& D, const void* xs, const void* vs, con
 
 template <typename T, int DD>
 lsh_status launch_attn_simt(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
-                            const float* invnorm, float* out_s, float* lse_s, cudaStream_t st) {
+                            const float* invnorm, T* out_s, float* lse_s, cudaStream_t st) {
   if (D.m <= 16) return launch_attn_simt_q<T, DD, 2>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
   if (D.m <= 32) return launch_attn_simt_q<T, DD, 4>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
   if (D.m <= 64) return launch_attn_simt_q<T, DD, 8>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
@@ -309,19 +309,19 @@ lsh_status launch_attn_tc_k(const CUtensorMap& tmx, const CUtensorMap& tmv,
 }
 
 lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
-                          const float* invnorm, float* out_r, float* lse, WsHeader* hdr,
+                          const float* invnorm, void* out_r, float* lse, WsHeader* hdr,
                           cudaStream_t st) {
   CUtensorMap tmx, tmv, tmo;
   const uint64_t rows = (uint64_t)D.S * D.n;
   if (!make_tmap_bf16_2d(&tmx, xs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys) ||
       !make_tmap_bf16_2d(&tmv, vs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys) ||
-      !make_tmap_f32_2d(&tmo, out_r, D.d, rows, (uint64_t)D.d * 4, 32, 32))
+      !make_tmap_bf16_2d(&tmo, out_r, D.d, rows, (uint64_t)D.d * 2, 64, 32))
     return LSH_ERR_CUDA;
   AttnTcArgs a;
   a.invnorm = invnorm;
   a.perm = perm;
   a.vs = static_cast<const __nv_bfloat16*>(vs);
-  a.out_r = out_r;
+  a.out_r = static_cast<__nv_bfloat16*>(out_r);
   a.lse = lse;
   a.hdr = hdr;
   a.n = D.n;
@@ -340,10 +340,11 @@ lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const i
 }
 
 template <typename T, int DD>
-lsh_status launch_merge(const Dims& D, const int32_t* inv, const float* lse, const float* out_r,
+lsh_status launch_merge(const Dims& D, const int32_t* inv, const float* lse, const T* out_r,
                         void* out, cudaStream_t st) {
   const int64_t total = D.BH * D.n;
-  const unsigned blocks = (unsigned)((total + kMergeWarps - 1) / kMergeWarps);
+  const int64_t per_block = kMergeWarps * 32 / (DD * (int)sizeof(T) / 16);  // positions
+  const unsigned blocks = (unsigned)((total + per_block - 1) / per_block);
   k_merge<T, DD><<<blocks, kMergeWarps * 32, 0, st>>>(inv, lse, out_r, static_cast<T*>(out), D.n,
                                                         D.rounds, total);
   return last_cuda();
@@ -369,7 +370,7 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
   float* invnorm = at<float>(ws, L.invnorm);
   void* xs = at<unsigned char>(ws, L.xs);
   void* vs = at<unsigned char>(ws, L.vs);
-  float* out_r = at<float>(ws, L.out_s);  // each round's output rows, slot order
+  T* out_r = at<T>(ws, L.out_s);  // each round's output rows, slot order
   if ((s = launch_sort<T>(D, buckets, x, v, perm, inv, xs, vs, invnorm, at<int32_t>(ws, L.hist),
                           hdr, st, ev)) != LSH_OK)
     return s;

@@ -7,10 +7,12 @@
 // round r at a position, LSE = logsumexp_r lse_r and
 //   out = sum_r exp(lse_r - LSE) * o_r,
 // i.e. one softmax over the union of the rounds' candidate lists.
-// One warp per (batch, head, position): lane r reads lse_r and slot_r (two
-// independent loads), the weights come from a warp max and sum, then every
-// round's fp32 row is loaded (four loads in flight before the sums) and the
-// output row is written once.
+// A group of G = D * sizeof(T) / 16 lanes merges one (batch, head,
+// position): lane j of the group owns the 16-byte piece j of every row. The
+// group's lanes read the rounds' lse (by position) and slots (inv) (lane j
+// takes rounds j, j + G, ...), the weights come from shuffles inside the
+// group, every round's row piece is loaded (four in flight before the sums)
+// and the output piece is written once.
 #pragma once
 
 #include "common.cuh"
@@ -19,66 +21,120 @@ namespace lsh {
 
 constexpr int kMergeWarps = 8;
 
-// grid ceil(BH * n / 8), block 256.
+template <int G>
+__device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+template <int G>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// 16 bytes of T as fp32.
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& a, float (&f)[16 / sizeof(T)]) {
+  if constexpr (sizeof(T) == 4) {
+    f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y);
+    f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+  } else {  // bf16: the high half of each 32-bit word is the later element
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[2 * k] = __uint_as_float(w[k] << 16);
+      f[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  }
+}
+
+// grid ceil(BH * n / (8 * 32 / G)), block 256.
 // inv, lse [BH][rounds][n] in position order; out_r [BH][rounds][n][D] in
-// slot order; out [BH][n][D] in T.
+// slot order and out [BH][n][D], both in T.
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeWarps * 32)
     k_merge(const int32_t* __restrict__ inv, const float* __restrict__ lse,
-            const float* __restrict__ out_r, T* __restrict__ out, int n, int rounds,
+            const T* __restrict__ out_r, T* __restrict__ out, int n, int rounds,
             int64_t total) {
-  const int lane = threadIdx.x & 31;
-  const int64_t item = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
-  if (item >= total) return;
-  const int64_t bh = item / n;
-  const int pos = (int)(item % n);
-  const float* segs = out_r + bh * rounds * (int64_t)n * D;  // round 0 of this (b, h)
+  constexpr int G = D * (int)sizeof(T) / 16;  // lanes per position: 8, 16 or 32
+  constexpr int EPV = 16 / (int)sizeof(T);    // elements per lane
+  constexpr int RPL = (16 + G - 1) / G;       // rounds per lane (rounds <= 16)
+  static_assert(G == 8 || G == 16 || G == 32, "a row is 128, 256 or 512 bytes");
+  static_assert(RPL <= 2, "the shuffles below pick one of at most two rounds per lane");
+  const int lane = threadIdx.x & 31, gl = lane % G, g0 = lane - gl;
+  const int64_t item =
+      ((int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5)) * (32 / G) + lane / G;
+  const bool valid = item < total;
+  const int64_t bh = valid ? item / n : 0;
+  const int pos = valid ? (int)(item % n) : 0;
 
   // w_r = exp(lse_r - mx) / sum_r' exp(lse_r' - mx). Forming logsumexp
   // first would round it to the fp32 grid near |lse| = 1e5 (self-only rows),
   // where the spacing is 1/128.
-  float l = -INFINITY;
-  int slot = 0;
-  if (lane < rounds) {
-    l = lse[(bh * rounds + lane) * (int64_t)n + pos];
-    slot = inv[(bh * rounds + lane) * (int64_t)n + pos];
+  float l[RPL], e[RPL];
+  int slot[RPL];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < RPL; ++k) {
+    const int r = gl + k * G;
+    l[k] = -INFINITY;
+    slot[k] = 0;
+    if (valid && r < rounds) {
+      l[k] = lse[(bh * rounds + r) * (int64_t)n + pos];
+      slot[k] = inv[(bh * rounds + r) * (int64_t)n + pos];
+    }
+    mx = fmaxf(mx, l[k]);
   }
-  const float mx = warp_max(l);
-  const float e = lane < rounds ? expf(l - mx) : 0.f;
-  const float w = e / warp_sum(e);
+  mx = group_max<G>(mx);
+  float es = 0.f;
+#pragma unroll
+  for (int k = 0; k < RPL; ++k) {
+    e[k] = gl + k * G < rounds ? expf(l[k] - mx) : 0.f;
+    es += e[k];
+  }
+  const float rs = 1.0f / group_sum<G>(es);
 
-  constexpr int DL = D / 32;  // dims per lane: 2 or 4
-  float acc[DL];
+  const T* segs = out_r + bh * rounds * (int64_t)n * D + gl * EPV;  // round 0 of this (b, h)
+  float acc[EPV];
 #pragma unroll
-  for (int k = 0; k < DL; ++k) acc[k] = 0.f;
+  for (int k = 0; k < EPV; ++k) acc[k] = 0.f;
   for (int r0 = 0; r0 < rounds; r0 += 4) {
-    float v[4][DL];
+    uint4 v[4];
+    float wr[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int sr = __shfl_sync(0xffffffffu, slot, (r0 + i) & 31);
-      const float* row = segs + ((int64_t)(r0 + i) * n + sr) * D + lane * DL;
-      if (r0 + i < rounds) {
-        if constexpr (DL == 4) {
-          const float4 a = *reinterpret_cast<const float4*>(row);
-          v[i][0] = a.x; v[i][1] = a.y; v[i][2] = a.z; v[i][3] = a.w;
-        } else {
-          const float2 a = *reinterpret_cast<const float2*>(row);
-          v[i][0] = a.x; v[i][1] = a.y;
-        }
-      }
+      const int r = r0 + i;  // uniform over the warp
+      const int k = r / G, src = g0 + r % G;
+      const int sr = __shfl_sync(0xffffffffu, k == 0 ? slot[0] : slot[RPL - 1], src);
+      wr[i] = __shfl_sync(0xffffffffu, k == 0 ? e[0] : e[RPL - 1], src) * rs;
+      if (valid && r < rounds)
+        v[i] = *reinterpret_cast<const uint4*>(segs + ((int64_t)r * n + sr) * D);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float wr = __shfl_sync(0xffffffffu, w, (r0 + i) & 31);
-      if (r0 + i < rounds) {
+      if (valid && r0 + i < rounds) {
+        float f[EPV];
+        unpack16<T>(v[i], f);
 #pragma unroll
-        for (int k = 0; k < DL; ++k) acc[k] = fmaf(wr, v[i][k], acc[k]);
+        for (int k = 0; k < EPV; ++k) acc[k] = fmaf(wr[i], f[k], acc[k]);
       }
     }
   }
-  T* o = out + item * D + lane * DL;
+  if (!valid) return;
+  T* o = out + item * D + gl * EPV;
+  if constexpr (sizeof(T) == 4) {
+    *reinterpret_cast<float4*>(o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  } else {
+    uint32_t w[4];
 #pragma unroll
-  for (int k = 0; k < DL; ++k) o[k] = Elem<T>::from_f(acc[k]);
+    for (int k = 0; k < 4; ++k) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * k], acc[2 * k + 1]);
+      w[k] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(o) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 }  // namespace lsh
