@@ -58,6 +58,15 @@ struct AttnTcArgs {
   int64_t pairs_per_cta;
 };
 
+// 2^x by the hardware's approximate base-2 exponential (relative error near
+// 2^-22, results below 2^-126 flushed to zero). The arguments here are <= 0
+// (logit minus an upper bound) and the results are rounded to bf16.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -263,17 +272,19 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         tmem_ld32(ts + wcol + b * 32, v);
         tmem_wait_ld();
         uint32_t pk[16];
+        const float4* kt4 = reinterpret_cast<const float4*>(kt + wcol + b * 32);
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float2 t0 = kt[wcol + b * 32 + c];
-          const float2 t1 = kt[wcol + b * 32 + c + 1];
-          const float l0 = fmaf(__uint_as_float(v[c]), t0.x, -bound);
-          const float l1 = fmaf(__uint_as_float(v[c + 1]), t1.x, -bound);
-          const float e0 = visible(__float_as_int(t0.y)) ? exp2f(l0) : 0.f;
-          const float e1 = visible(__float_as_int(t1.y)) ? exp2f(l1) : 0.f;
-          sum0 += e0;
-          sum1 += e1;
-          pk[c >> 1] = pack_bf16x2(e0, e1);
+          const float4 t = kt4[c >> 1];  // (scale, position) of keys c and c + 1
+          // every exponent is computed, then invisible keys are masked: no
+          // divergent branch per key
+          const float e0 = ex2_approx(fmaf(__uint_as_float(v[c]), t.x, -bound));
+          const float e1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), t.z, -bound));
+          const float p0 = visible(__float_as_int(t.y)) ? e0 : 0.f;
+          const float p1 = visible(__float_as_int(t.w)) ? e1 : 0.f;
+          sum0 += p0;
+          sum1 += p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
         }
         // P column c holds keys 2c, 2c+1: chunk b lands in columns
         // [wcol/2 + 16b, wcol/2 + 16b + 16), behind every S column still unread
