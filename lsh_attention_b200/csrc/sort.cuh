@@ -60,17 +60,32 @@ __global__ void __launch_bounds__(256)
 }
 
 // grid (segments), block 1024: in-place exclusive scan of len ints per segment.
+// Each thread scans a contiguous run of kScanPer counts, all loaded before
+// any is used (sixteen-byte loads when the segment is 16-byte aligned), so a
+// segment of up to 32K counts costs one load round trip and one block scan.
+constexpr int kScanPer = 32;
 __global__ void __launch_bounds__(1024) k_sort_scan(int32_t* __restrict__ hist, int len) {
   __shared__ int32_t wsum[32];
   int32_t* h = hist + (int64_t)blockIdx.x * len;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool vec = (len & 3) == 0;  // then every run of 4 starts 16-byte aligned
   int32_t carry = 0;
-  for (int base = 0; base < len; base += 4 * 1024) {
-    const int i0 = base + 4 * threadIdx.x;
-    int32_t v[4];
+  for (int base = 0; base < len; base += kScanPer * 1024) {
+    const int i0 = base + kScanPer * threadIdx.x;
+    int32_t v[kScanPer];
+    if (vec && i0 + kScanPer <= len) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = (i0 + k < len) ? h[i0 + k] : 0;
-    const int32_t local = v[0] + v[1] + v[2] + v[3];
+      for (int k = 0; k < kScanPer; k += 4) {
+        const int4 q = *reinterpret_cast<const int4*>(h + i0 + k);
+        v[k] = q.x; v[k + 1] = q.y; v[k + 2] = q.z; v[k + 3] = q.w;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < kScanPer; ++k) v[k] = (i0 + k < len) ? h[i0 + k] : 0;
+    }
+    int32_t local = 0;
+#pragma unroll
+    for (int k = 0; k < kScanPer; ++k) local += v[k];
     int32_t incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -91,9 +106,19 @@ __global__ void __launch_bounds__(1024) k_sort_scan(int32_t* __restrict__ hist, 
     __syncthreads();
     int32_t run = carry + (warp > 0 ? wsum[warp - 1] : 0) + incl - local;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      if (i0 + k < len) h[i0 + k] = run;
-      run += v[k];
+    for (int k = 0; k < kScanPer; ++k) {
+      const int32_t c = v[k];
+      v[k] = run;
+      run += c;
+    }
+    if (vec && i0 + kScanPer <= len) {
+#pragma unroll
+      for (int k = 0; k < kScanPer; k += 4)
+        *reinterpret_cast<int4*>(h + i0 + k) = make_int4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < kScanPer; ++k)
+        if (i0 + k < len) h[i0 + k] = v[k];
     }
     carry += wsum[31];
     __syncthreads();
