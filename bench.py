@@ -40,10 +40,11 @@ STAGES = ("hash", "sort_gather", "chunk_attention", "unsort_merge")
 KERNELS = lb.PROFILE_KERNELS
 KERNEL_STAGE = {"hash_prep": "hash", "hash_mma": "hash", "hash_refine": "hash",
                 "sort_hist": "sort_gather", "sort_scan": "sort_gather",
-                "sort_scatter_gather": "sort_gather", "chunk_attention": "chunk_attention",
+                "sort_rank": "sort_gather", "row_gather": "sort_gather",
+                "chunk_attention": "chunk_attention",
                 "unsort_merge": "unsort_merge"}
 # the kernel that carries a stage's algorithmic work
-STAGE_KERNEL = {"hash": "hash_mma", "sort_gather": "sort_scatter_gather",
+STAGE_KERNEL = {"hash": "hash_mma", "sort_gather": "row_gather",
                 "chunk_attention": "chunk_attention", "unsort_merge": "unsort_merge"}
 # DRAM bytes (read + write) per launch from one ncu capture of the long-64k
 # workload, valid only while the kernel's source file is unchanged (sha256
@@ -51,19 +52,21 @@ STAGE_KERNEL = {"hash": "hash_mma", "sort_gather": "sort_scatter_gather",
 NCU_TRAFFIC = {
     "hash_prep": {"bytes": 532000, "file": "hash_tc.cuh",
         "sha256": "684e370eca8f9f6eab6507cda92eff0e6f320859492c5b7d1d373eb0080708a5"},
-    "hash_mma": {"bytes": 144067000, "file": "hash_tc.cuh",
+    "hash_mma": {"bytes": 143350000, "file": "hash_tc.cuh",
         "sha256": "684e370eca8f9f6eab6507cda92eff0e6f320859492c5b7d1d373eb0080708a5"},
     "hash_refine": {"bytes": 2050000, "file": "hash_tc.cuh",
         "sha256": "684e370eca8f9f6eab6507cda92eff0e6f320859492c5b7d1d373eb0080708a5"},
     "sort_hist": {"bytes": 8393000, "file": "sort.cuh",
-        "sha256": "bb18c7ce75121f48157bba07d459db2fb295f4bb5d321eeaf0abcc010ec71cb7"},
-    "sort_scan": {"bytes": 4199000, "file": "sort.cuh",
-        "sha256": "bb18c7ce75121f48157bba07d459db2fb295f4bb5d321eeaf0abcc010ec71cb7"},
-    "sort_scatter_gather": {"bytes": 1409771000, "file": "sort_tma.cuh",
-        "sha256": "5f1e2222ff32e16d9196fd996834ecd1cfd0ed703df3ba11f6338726720cdce7"},
-    "chunk_attention": {"bytes": 1654679000, "file": "attn_tc.cuh",
-        "sha256": "bad5498d5272605d7327ada9bc907ae21333a470122a2e0897b413a37963efad"},
-    "unsort_merge": {"bytes": 673733000, "file": "merge.cuh",
+        "sha256": "37325b5c5f6026dbc17d72ab5ec36f8c8345a74c9c0f39a902008b1d1a7725bf"},
+    "sort_scan": {"bytes": 4204000, "file": "sort.cuh",
+        "sha256": "37325b5c5f6026dbc17d72ab5ec36f8c8345a74c9c0f39a902008b1d1a7725bf"},
+    "sort_rank": {"bytes": 12602000, "file": "sort.cuh",
+        "sha256": "37325b5c5f6026dbc17d72ab5ec36f8c8345a74c9c0f39a902008b1d1a7725bf"},
+    "row_gather": {"bytes": 1514572000, "file": "gather.cuh",
+        "sha256": "e6ed6996ab9b55d7b4ab341085d7fa0a4c9c38b1532727b5bb8fad26bde2238a"},
+    "chunk_attention": {"bytes": 1652833000, "file": "attn_tc.cuh",
+        "sha256": "662aea74507cfaa09642c7e3d073502e380987346a7690e33e3af2093889c234"},
+    "unsort_merge": {"bytes": 673753000, "file": "merge.cuh",
         "sha256": "434e0ca452f2adcc23b4642755cd266872e0601d79c6d2c1704dabe29dfd4805"},
 }
 
@@ -90,7 +93,10 @@ def algorithmic(w: I.Workload) -> dict:
     return {
         "hash": {"bytes": X + Rn * w.d * (w.n_buckets // 2) * E + 4 * T * Rn,
                  "flops": 2 * T * w.d * (w.n_buckets // 2) * Rn},
-        "sort_gather": {"bytes": 4 * T * Rn + 2 * X * Rn + 2 * X * Rn + 8 * T * Rn, "flops": 0},
+        # the row gather, which carries the stage: perm in, x and v once per
+        # (batch, head) (the rounds share them through L2), xs and vs rows
+        # out, 1/||x|| out (ranks and histograms: ~1% more)
+        "sort_gather": {"bytes": 4 * T * Rn + 2 * X + 2 * X * Rn + 4 * T * Rn, "flops": 0},
         "chunk_attention": {"bytes": 2 * X * Rn + 4 * T * Rn + T * Rn * w.d * E + 4 * T * Rn,
                             "flops": 8 * m * w.d * T * Rn},
         "unsort_merge": {"bytes": T * Rn * (E * w.d + 8) + X, "flops": 0},
@@ -405,8 +411,8 @@ def run_ours(args, w):
 
 def launches_per_forward(buckets_given: bool) -> int:
     # hash: rotation transpose, projection/argmax, fp64 re-decision (3); sort:
-    # histogram, scan, rank/scatter/gather (3); attention (1); merge (1)
-    return (0 if buckets_given else 3) + 3 + 1 + 1
+    # histogram, scan, ranks, row gather (4); attention (1); merge (1)
+    return (0 if buckets_given else 3) + 4 + 1 + 1
 
 
 def traffic_of(kernel: str):

@@ -124,15 +124,15 @@ lsh_status lsh_attn_forward(const lsh_attn_desc *desc, const void *x, const void
                             void *workspace, size_t workspace_bytes, void *stream);
 
 /* Number of events lsh_attn_forward_profiled records. */
-#define LSH_ATTN_PROFILE_EVENTS 9
+#define LSH_ATTN_PROFILE_EVENTS 10
 
 /* lsh_attn_forward that also records the caller's CUDA events on `stream`
  * at every kernel boundary, for timing each kernel on the device:
  *   [0] start               [1] after the rotation transpose of the hash
  *   [2] after the projection / argmax kernel  [3] after the fp64 re-decision
  *   [4] after the bucket histograms  [5] after their scan
- *   [6] after the stable ranks, perm/inv and row gather
- *   [7] after the chunked attention  [8] after the un-sort and round merge
+ *   [6] after the stable ranks (perm/inv)  [7] after the row gather
+ *   [8] after the chunked attention  [9] after the un-sort and round merge
  * A kernel that does not run for this problem (caller-supplied buckets, the
  * fp64 hash) leaves consecutive events with nothing between them.
  * `events` points to LSH_ATTN_PROFILE_EVENTS cudaEvent_t handles created by

@@ -9,11 +9,11 @@
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
+#include "gather.cuh"
 #include "hash_exact.cuh"
 #include "hash_tc.cuh"
 #include "merge.cuh"
 #include "sort.cuh"
-#include "sort_tma.cuh"
 #include "tma_host.cuh"
 
 namespace {
@@ -237,34 +237,27 @@ lsh_status launch_sort(const Dims& D, const int32_t* buckets, const void* x, con
   if ((s = mark(ev, 4, st)) != LSH_OK) return s;
   k_sort_scan<<<(unsigned)D.S, 1024, 0, st>>>(hist, D.nb * D.tiles);
   if ((s = mark(ev, 5, st)) != LSH_OK) return s;
-  if (xs != nullptr) {  // ranks + row gather, rows streamed by TMA
-    const SortGatherPlan gp = sort_gather_plan(D.nb, D.d, (int)sizeof(T));
-    CUtensorMap tmx, tmv;
-    const uint64_t rows = (uint64_t)D.BH * D.n;
-    if (!make_tmap_plain_2d(&tmx, x, (int)sizeof(T), D.d, rows, D.d, gp.chunk_rows) ||
-        !make_tmap_plain_2d(&tmv, v, (int)sizeof(T), D.d, rows, D.d, gp.chunk_rows))
-      return LSH_ERR_CUDA;
-    auto kern = k_sort_gather_tma<T>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gp.smem) !=
-        cudaSuccess)
-      return LSH_ERR_CUDA;
-    kern<<<grid, gp.nw * 32, gp.smem, st>>>(tmx, tmv, buckets, hist, perm, inv,
-                                             static_cast<T*>(xs), static_cast<T*>(vs), invnorm,
-                                             D.n, D.d, D.nb, D.rounds, D.tiles, gp.chunk_rows, hdr);
-  } else {  // ranks only
+  {  // stable ranks: perm and inv
     const int nw = sort_warps(D.nb);
     const size_t smem = sizeof(int32_t) * (size_t)nw * D.nb;
-    auto kern = k_sort_scatter<T>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(k_sort_rank, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
       return LSH_ERR_CUDA;
-    kern<<<grid, nw * 32, smem, st>>>(buckets, hist, static_cast<const T*>(x),
-                                       static_cast<const T*>(v), perm, inv, static_cast<T*>(xs),
-                                       static_cast<T*>(vs), invnorm, D.n, D.d, D.nb, D.rounds,
-                                       D.tiles);
+    k_sort_rank<<<grid, nw * 32, smem, st>>>(buckets, hist, perm, inv, D.n, D.nb, D.tiles);
   }
   if ((s = last_cuda()) != LSH_OK) return s;
-  return mark(ev, 6, st);
+  if ((s = mark(ev, 6, st)) != LSH_OK) return s;
+  if (xs != nullptr) {  // the rows in slot order, with 1/||x||
+    const int64_t blocks =
+        D.BH * (int64_t)((D.n + kGatherSlots - 1) / kGatherSlots) * D.rounds;
+    if (blocks > INT32_MAX) return LSH_ERR_UNSUPPORTED;
+    auto kern = D.d == 64 ? k_gather_rows<T, 64> : k_gather_rows<T, 128>;
+    kern<<<(unsigned)blocks, kGatherWarps * 32, 0, st>>>(
+        perm, static_cast<const T*>(x), static_cast<const T*>(v), static_cast<T*>(xs),
+        static_cast<T*>(vs), invnorm, D.n, D.rounds);
+  }
+  if ((s = last_cuda()) != LSH_OK) return s;
+  return mark(ev, 7, st);
 }
 
 template <typename T, int DD, int QPW>
@@ -380,11 +373,11 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
     s = D.d == 64 ? launch_attn_simt<T, 64>(D, xs, vs, perm, invnorm, out_r, lse, st)
                   : launch_attn_simt<T, 128>(D, xs, vs, perm, invnorm, out_r, lse, st);
   if (s != LSH_OK) return s;
-  if ((s = mark(ev, 7, st)) != LSH_OK) return s;
+  if ((s = mark(ev, 8, st)) != LSH_OK) return s;
   s = D.d == 64 ? launch_merge<T, 64>(D, inv, lse, out_r, out, st)
                 : launch_merge<T, 128>(D, inv, lse, out_r, out, st);
   if (s != LSH_OK) return s;
-  return mark(ev, 8, st);
+  return mark(ev, 9, st);
 }
 
 }  // namespace

@@ -14,13 +14,15 @@
 #include <mutex>
 
 #include "lsh_attn.h"
-// This file is a translation unit of its own: the two non-template sort
-// kernels get file-local names so they do not collide with lsh_attn.cu's.
+// This file is a translation unit of its own: the sort kernels get file-local
+// names so they do not collide with lsh_attn.cu's.
 #define k_sort_hist k_sort_hist_noalloc
 #define k_sort_scan k_sort_scan_noalloc
+#define k_sort_rank k_sort_rank_noalloc
 #include "sort.cuh"
 #undef k_sort_hist
 #undef k_sort_scan
+#undef k_sort_rank
 
 namespace {
 
@@ -89,11 +91,10 @@ extern "C" lsh_status lsh_attn_sort_noalloc(const lsh_attn_desc* desc, const int
   k_sort_scan_noalloc<<<(unsigned)segs, 1024, 0, st>>>(hist, q.n_buckets * tiles);
   const int nw = sort_warps(q.n_buckets);
   const size_t smem = sizeof(int32_t) * (size_t)nw * q.n_buckets;
-  auto kern = k_sort_scatter<__nv_bfloat16>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(k_sort_rank_noalloc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
     return LSH_ERR_CUDA;
-  kern<<<grid, nw * 32, smem, st>>>(buckets, hist, nullptr, nullptr, perm, inv, nullptr, nullptr,
-                                     nullptr, q.n, 64, q.n_buckets, q.rounds, tiles);
+  k_sort_rank_noalloc<<<grid, nw * 32, smem, st>>>(buckets, hist, perm, inv, q.n, q.n_buckets,
+                                                   tiles);
   return cudaGetLastError() == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
 }

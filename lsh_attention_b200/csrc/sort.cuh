@@ -5,12 +5,12 @@
 // bucket, and inside a bucket by position. Positions are already in order, so
 // slot(i) = #{j : b_j < b_i} + #{j < i : b_j = b_i}. Three kernels compute it
 // without a global sort:
-//   k_sort_hist     per-(segment, tile) bucket histograms, warp-aggregated
-//   k_sort_scan     exclusive scan of each segment's [bucket][tile] counts
-//   k_sort_scatter  per-warp counts inside the tile, stable ranks from
-//                   __match_any_sync, perm/inv writes, and the row gather
-// A segment is one (batch, head, round); a tile is kSortWarps(nb) warps of
-// kSortSub tokens each.
+//   k_sort_hist   per-(segment, tile) bucket histograms, warp-aggregated
+//   k_sort_scan   exclusive scan of each segment's [bucket][tile] counts
+//   k_sort_rank   per-warp counts inside the tile, stable ranks from
+//                 __match_any_sync, perm/inv writes
+// (the rows follow in slot order: k_gather_rows). A segment is one (batch,
+// head, round); a tile is sort_warps(nb) warps of kSortSub tokens each.
 #pragma once
 
 #include "common.cuh"
@@ -125,56 +125,11 @@ __global__ void __launch_bounds__(1024) k_sort_scan(int32_t* __restrict__ hist, 
   }
 }
 
-// Copy 32 rows (one per lane's token) of x and v into sorted order and write
-// each row's inverse key norm. Lane L holds the slot of token t0 + L.
-template <typename T>
-__device__ __forceinline__ void gather_rows(const T* __restrict__ xg, const T* __restrict__ vg,
-                                            int t0, int valid_count, int slot_mine, int d,
-                                            T* __restrict__ xs, T* __restrict__ vs,
-                                            float* __restrict__ invnorm) {
-  const int lane = threadIdx.x & 31;
-  const int cpr = d * (int)sizeof(T) / 16;  // 16-byte chunks per row (8..32)
-  const int rpp = 32 / cpr > 0 ? 32 / cpr : 1;  // rows per pass
-  const int lanes_per_row = cpr < 32 ? cpr : 32;
-  const int iters_per_row = cpr / lanes_per_row;  // 1, or 2 for 512-byte rows
-#pragma unroll 4
-  for (int r0 = 0; r0 < 32; r0 += rpp) {
-    const int ri = r0 + lane / lanes_per_row;
-    const int c = lane % lanes_per_row;
-    const int slot = __shfl_sync(0xffffffffu, slot_mine, ri & 31);
-    const bool ok = ri < valid_count;
-    float ss = 0.f;
-    if (ok) {
-      const uint4* xr = reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + ri) * d);
-      const uint4* vr = reinterpret_cast<const uint4*>(vg + (int64_t)(t0 + ri) * d);
-      uint4* xo = reinterpret_cast<uint4*>(xs + (int64_t)slot * d);
-      uint4* vo = reinterpret_cast<uint4*>(vs + (int64_t)slot * d);
-      for (int it = 0; it < iters_per_row; ++it) {
-        const int cc = c + it * lanes_per_row;
-        const uint4 a = __ldg(xr + cc);
-        const uint4 b = __ldg(vr + cc);
-        xo[cc] = a;
-        vo[cc] = b;
-        float f[Vec16<T>::N];
-        Vec16<T>::unpack(a, f);
-#pragma unroll
-        for (int k = 0; k < Vec16<T>::N; ++k) ss = fmaf(f[k], f[k], ss);
-      }
-    }
-    for (int o = lanes_per_row / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (ok && c == 0) invnorm[slot] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
-  }
-}
-
-// grid (tiles, segments), block sort_warps(nb) * 32.
-// hist: scanned offsets [seg][nb][tiles]. perm, inv, invnorm: [seg][n];
-// xs, vs: [seg][n][d] (skipped when xs == nullptr). x, v: [BH][n][d].
-template <typename T>
+// grid (tiles, segments), block sort_warps(nb) * 32, shared nw * nb ints.
+// hist: scanned offsets [seg][nb][tiles]. perm, inv: [seg][n].
 __global__ void __launch_bounds__(512)
-    k_sort_scatter(const int32_t* __restrict__ buckets, const int32_t* __restrict__ hist,
-                   const T* __restrict__ x, const T* __restrict__ v, int32_t* __restrict__ perm,
-                   int32_t* __restrict__ inv, T* __restrict__ xs, T* __restrict__ vs,
-                   float* __restrict__ invnorm, int n, int d, int nb, int rounds, int tiles) {
+    k_sort_rank(const int32_t* __restrict__ buckets, const int32_t* __restrict__ hist,
+                int32_t* __restrict__ perm, int32_t* __restrict__ inv, int n, int nb, int tiles) {
   extern __shared__ int32_t base[];  // [warps][nb]
   const int seg = blockIdx.y, tl = blockIdx.x;
   const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -207,10 +162,7 @@ __global__ void __launch_bounds__(512)
     }
   }
   __syncthreads();
-  // 3) stable ranks, perm / inv, and the gather
-  const int64_t bh = seg / rounds;
-  const T* xg = x + bh * (int64_t)n * d;
-  const T* vg = v + bh * (int64_t)n * d;
+  // 3) stable ranks, perm / inv
   const int64_t so = (int64_t)seg * n;
   for (int s0 = wstart; s0 < wend; s0 += 32) {
     const int t = s0 + lane;
@@ -225,8 +177,6 @@ __global__ void __launch_bounds__(512)
       perm[so + slot] = t;
       inv[so + t] = slot;
     }
-    if (xs != nullptr)
-      gather_rows<T>(xg, vg, s0, wend - s0, slot, d, xs + so * d, vs + so * d, invnorm + so);
   }
 }
 
