@@ -40,13 +40,22 @@ __global__ void __launch_bounds__(256)
   const int start = tl * tile, end = min(n, start + tile);
   const int32_t* bk = buckets + (int64_t)seg * n;
   const int lane = threadIdx.x & 31;
-  for (int base = start; base < end; base += blockDim.x) {
-    const int t = base + threadIdx.x;
+  // every id of the tile is loaded before the first is counted (a tile is at
+  // most kSortSub * 8 = 2048 tokens, 8 per thread of the 256)
+  constexpr int kPer = 8;
+  int raw[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int t = start + i * 256 + threadIdx.x;
+    raw[i] = t < end ? bk[t] : 0;
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int t = start + i * 256 + threadIdx.x;
     int b = -1;
     if (t < end) {
-      const int raw = bk[t];
-      b = clamp_bucket(raw, nb);
-      if (b != raw) {
+      b = clamp_bucket(raw[i], nb);
+      if (b != raw[i]) {
         atomicAdd(&hdr->bad_bucket_ids, 1u);
         record_status(hdr, 6u /* LSH_ERR_DEVICE */);
       }
@@ -142,10 +151,18 @@ __global__ void __launch_bounds__(512)
   const int32_t* bk = buckets + (int64_t)seg * n;
   int32_t* mybase = base + warp * nb;
 
+  // this warp's ids, loaded once for both passes (-1 past the end)
+  constexpr int kSteps = kSortSub / 32;
+  int bks[kSteps];
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) {
+    const int t = wstart + 32 * i + lane;
+    bks[i] = t < wend ? clamp_bucket(bk[t], nb) : -1;
+  }
   // 1) per-warp counts of its sub-range
-  for (int s0 = wstart; s0 < wend; s0 += 32) {
-    const int t = s0 + lane;
-    const int b = t < wend ? clamp_bucket(bk[t], nb) : -1;
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) {
+    const int b = bks[i];
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
     if (b >= 0 && lane == __ffs(peers) - 1) mybase[b] += __popc(peers);
     __syncwarp();
@@ -164,9 +181,10 @@ __global__ void __launch_bounds__(512)
   __syncthreads();
   // 3) stable ranks, perm / inv
   const int64_t so = (int64_t)seg * n;
-  for (int s0 = wstart; s0 < wend; s0 += 32) {
-    const int t = s0 + lane;
-    const int b = t < wend ? clamp_bucket(bk[t], nb) : -1;
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) {
+    const int t = wstart + 32 * i + lane;
+    const int b = bks[i];
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
     int slot = 0;
     if (b >= 0) slot = mybase[b] + __popc(peers & lanemask_lt());
