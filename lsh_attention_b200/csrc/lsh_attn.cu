@@ -3,6 +3,8 @@
 #include "lsh_attn.h"
 
 #include <cuda_runtime.h>
+
+#include <algorithm>
 #include <stdint.h>
 #include <string.h>
 
@@ -337,7 +339,8 @@ lsh_status launch_merge(const Dims& D, const int32_t* inv, const float* lse, con
                         void* out, cudaStream_t st) {
   const int64_t total = D.BH * D.n;
   const int64_t per_block = kMergeWarps * 32 / (DD * (int)sizeof(T) / 16);  // positions
-  const unsigned blocks = (unsigned)((total + per_block - 1) / per_block);
+  const int64_t cap = (int64_t)kMergeCtasPerSm * sm_count();
+  const unsigned blocks = (unsigned)std::min<int64_t>((total + per_block - 1) / per_block, cap);
   k_merge<T, DD><<<blocks, kMergeWarps * 32, 0, st>>>(inv, lse, out_r, static_cast<T*>(out), D.n,
                                                         D.rounds, total);
   return last_cuda();
