@@ -52,22 +52,22 @@ STAGE_KERNEL = {"hash": "hash_mma", "sort_gather": "row_gather",
 NCU_TRAFFIC = {
     "hash_prep": {"bytes": 532000, "file": "hash_tc.cuh",
         "sha256": "684e370eca8f9f6eab6507cda92eff0e6f320859492c5b7d1d373eb0080708a5"},
-    "hash_mma": {"bytes": 143350000, "file": "hash_tc.cuh",
+    "hash_mma": {"bytes": 145299000, "file": "hash_tc.cuh",
         "sha256": "684e370eca8f9f6eab6507cda92eff0e6f320859492c5b7d1d373eb0080708a5"},
-    "hash_refine": {"bytes": 2050000, "file": "hash_tc.cuh",
+    "hash_refine": {"bytes": 2050999, "file": "hash_tc.cuh",
         "sha256": "684e370eca8f9f6eab6507cda92eff0e6f320859492c5b7d1d373eb0080708a5"},
-    "sort_hist": {"bytes": 8393000, "file": "sort.cuh",
-        "sha256": "37325b5c5f6026dbc17d72ab5ec36f8c8345a74c9c0f39a902008b1d1a7725bf"},
+    "sort_hist": {"bytes": 8399000, "file": "sort.cuh",
+        "sha256": "43310597a747f8b8ba4912eef7ba900a3bd625ec3c0600427c15a179e06518d0"},
     "sort_scan": {"bytes": 4204000, "file": "sort.cuh",
-        "sha256": "37325b5c5f6026dbc17d72ab5ec36f8c8345a74c9c0f39a902008b1d1a7725bf"},
-    "sort_rank": {"bytes": 12602000, "file": "sort.cuh",
-        "sha256": "37325b5c5f6026dbc17d72ab5ec36f8c8345a74c9c0f39a902008b1d1a7725bf"},
-    "row_gather": {"bytes": 1514572000, "file": "gather.cuh",
+        "sha256": "43310597a747f8b8ba4912eef7ba900a3bd625ec3c0600427c15a179e06518d0"},
+    "sort_rank": {"bytes": 12595000, "file": "sort.cuh",
+        "sha256": "43310597a747f8b8ba4912eef7ba900a3bd625ec3c0600427c15a179e06518d0"},
+    "row_gather": {"bytes": 1514832000, "file": "gather.cuh",
         "sha256": "e6ed6996ab9b55d7b4ab341085d7fa0a4c9c38b1532727b5bb8fad26bde2238a"},
-    "chunk_attention": {"bytes": 1652833000, "file": "attn_tc.cuh",
+    "chunk_attention": {"bytes": 1652675000, "file": "attn_tc.cuh",
         "sha256": "662aea74507cfaa09642c7e3d073502e380987346a7690e33e3af2093889c234"},
-    "unsort_merge": {"bytes": 673753000, "file": "merge.cuh",
-        "sha256": "434e0ca452f2adcc23b4642755cd266872e0601d79c6d2c1704dabe29dfd4805"},
+    "unsort_merge": {"bytes": 672961000, "file": "merge.cuh",
+        "sha256": "f313dd4622da3353060cb7b84324a099bfef2be35a4e693135b8674f34cd17db"},
 }
 
 
