@@ -149,6 +149,17 @@ lsh_status lsh_attn_get_device_status(const void *workspace, void *stream);
 /* Synchronise `stream` and copy the workspace counters into *diag. */
 lsh_status lsh_attn_get_diag(const void *workspace, void *stream, lsh_attn_diag *diag);
 
+/* Self-test of the bounded waits every kernel uses: clears the workspace
+ * status word, then launches one CTA that waits on an mbarrier nothing
+ * arrives at, with a limit of `limit_us` microseconds (1 .. 2000000) instead
+ * of the kernels' 2 s. The wait gives up, the kernel records LSH_ERR_TIMEOUT
+ * in the status word and returns, and the stream stays usable: read the
+ * status with lsh_attn_get_device_status. `workspace` needs at least 256
+ * bytes. Returns LSH_ERR_INVALID_ARG for a null workspace, too small a size
+ * or a limit out of range (nothing is launched then). */
+lsh_status lsh_attn_selftest_wait_timeout(void *workspace, size_t workspace_bytes,
+                                          uint32_t limit_us, void *stream);
+
 /* Size of the device-resident scratch of lsh_attn_sort_noalloc (8 MiB). */
 #define LSH_ATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
 

@@ -25,7 +25,7 @@ _DTYPES = {torch.float32: LSH_F32, torch.bfloat16: LSH_BF16}
 #: every symbol the header declares
 EXPORTS = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_forward",
            "lsh_attn_forward_profiled", "lsh_attn_get_device_status", "lsh_attn_get_diag",
-           "lsh_attn_sort_noalloc", "lsh_attn_status_string")
+           "lsh_attn_sort_noalloc", "lsh_attn_selftest_wait_timeout", "lsh_attn_status_string")
 
 
 class LshAttnDesc(ctypes.Structure):
@@ -72,6 +72,7 @@ def load() -> ctypes.CDLL:
             lib.lsh_attn_get_device_status.argtypes = [vp, vp]
             lib.lsh_attn_sort_noalloc.argtypes = [dp, vp, vp, vp]
             lib.lsh_attn_get_diag.argtypes = [vp, vp, ctypes.POINTER(LshAttnDiag)]
+            lib.lsh_attn_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
             lib.lsh_attn_status_string.argtypes = [ctypes.c_int]
             lib.lsh_attn_status_string.restype = ctypes.c_char_p
             for f in EXPORTS[:-1]:
@@ -247,3 +248,12 @@ def lsh_attn_get_diag(ws, stream=None) -> dict:
 
 def lsh_attn_get_device_status(ws, stream=None) -> int:
     return load().lsh_attn_get_device_status(_ptr(ws), _stream(stream))
+
+
+def lsh_attn_selftest_wait_timeout(ws, limit_us: int, stream=None) -> None:
+    """Launch the bounded-wait self-test on `ws` (a uint8 CUDA tensor of at
+    least 256 bytes): a wait that nothing completes gives up after
+    `limit_us` and records LSH_ERR_TIMEOUT (read it with
+    lsh_attn_get_device_status)."""
+    _check(load().lsh_attn_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(),
+                                                 int(limit_us), _stream(stream)))

@@ -115,6 +115,19 @@ lsh_status reset_header(void* ws, cudaStream_t st) {
   return cudaMemsetAsync(ws, 0, sizeof(WsHeader), st) == cudaSuccess ? LSH_OK : LSH_ERR_CUDA;
 }
 
+// One CTA waits on an mbarrier that nothing arrives at, with a short limit:
+// the wait gives up, the status word records the timeout, the kernel returns.
+__global__ void k_wait_selftest(WsHeader* hdr, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !sm100::mbar_wait(&bar, 0, limit_ns))
+    record_status(hdr, 5u /* LSH_ERR_TIMEOUT */);
+}
+
 // ---------------------------------------------------------------- launches
 // Profiling marks: the events of lsh_attn_forward_profiled, one per kernel
 // boundary (indices in lsh_attn.h).
@@ -241,7 +254,7 @@ lsh_status launch_sort(const Dims& D, const int32_t* buckets, const void* x, con
   if ((s = mark(ev, 5, st)) != LSH_OK) return s;
   {  // stable ranks: perm and inv
     const int nw = sort_warps(D.nb);
-    const size_t smem = sizeof(int32_t) * (size_t)nw * D.nb;
+    const size_t smem = sort_rank_smem(D.nb);
     if (cudaFuncSetAttribute(k_sort_rank, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return LSH_ERR_CUDA;
@@ -487,6 +500,17 @@ lsh_status lsh_attn_get_diag(const void* ws, void* stream, lsh_attn_diag* diag) 
   diag->bad_bucket_ids = h.bad_bucket_ids;
   diag->reserved = 0;
   return LSH_OK;
+}
+
+lsh_status lsh_attn_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us,
+                                          void* stream) {
+  if (!ws || ws_bytes < sizeof(WsHeader) || limit_us < 1 || limit_us > 2000000u)
+    return LSH_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  lsh_status s = reset_header(ws, st);
+  if (s != LSH_OK) return s;
+  k_wait_selftest<<<1, 32, 0, st>>>(static_cast<WsHeader*>(ws), (uint64_t)limit_us * 1000u);
+  return last_cuda();
 }
 
 lsh_status lsh_attn_get_device_status(const void* ws, void* stream) {

@@ -90,7 +90,7 @@ extern "C" lsh_status lsh_attn_sort_noalloc(const lsh_attn_desc* desc, const int
                                                                 tiles, hist, hdr);
   k_sort_scan_noalloc<<<(unsigned)segs, 1024, 0, st>>>(hist, q.n_buckets * tiles);
   const int nw = sort_warps(q.n_buckets);
-  const size_t smem = sizeof(int32_t) * (size_t)nw * q.n_buckets;
+  const size_t smem = sort_rank_smem(q.n_buckets);
   if (cudaFuncSetAttribute(k_sort_rank_noalloc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return LSH_ERR_CUDA;

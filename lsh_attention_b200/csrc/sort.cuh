@@ -134,22 +134,32 @@ __global__ void __launch_bounds__(1024) k_sort_scan(int32_t* __restrict__ hist, 
   }
 }
 
-// grid (tiles, segments), block sort_warps(nb) * 32, shared nw * nb ints.
+// Shared memory of k_sort_rank: the tile's offset of every bucket (int32)
+// and each warp's running count in the bucket inside the tile (16 bits: a
+// tile holds at most 2048 tokens).
+__host__ __device__ inline size_t sort_rank_smem(int nb) {
+  return sizeof(int32_t) * (size_t)nb + sizeof(uint16_t) * (size_t)sort_warps(nb) * nb;
+}
+
+// grid (tiles, segments), block sort_warps(nb) * 32, shared sort_rank_smem(nb).
 // hist: scanned offsets [seg][nb][tiles]. perm, inv: [seg][n].
-__global__ void __launch_bounds__(512)
+// Eight CTAs of 256 threads fit an SM, so a long-sequence launch is one wave.
+__global__ void __launch_bounds__(256, 8)
     k_sort_rank(const int32_t* __restrict__ buckets, const int32_t* __restrict__ hist,
                 int32_t* __restrict__ perm, int32_t* __restrict__ inv, int n, int nb, int tiles) {
-  extern __shared__ int32_t base[];  // [warps][nb]
+  extern __shared__ int32_t toff[];  // [nb], then uint16 [warps][nb]
   const int seg = blockIdx.y, tl = blockIdx.x;
   const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < nw * nb; i += blockDim.x) base[i] = 0;
+  uint16_t* cnt = reinterpret_cast<uint16_t*>(toff + nb);
+  uint32_t* cnt32 = reinterpret_cast<uint32_t*>(cnt);  // nb is even
+  for (int i = threadIdx.x; i < nw * nb / 2; i += blockDim.x) cnt32[i] = 0u;
   __syncthreads();
 
   const int tile = nw * kSortSub;
   const int wstart = tl * tile + warp * kSortSub;
   const int wend = min(n, wstart + kSortSub);
   const int32_t* bk = buckets + (int64_t)seg * n;
-  int32_t* mybase = base + warp * nb;
+  uint16_t* mycnt = cnt + warp * nb;
 
   // this warp's ids, loaded once for both passes (-1 past the end)
   constexpr int kSteps = kSortSub / 32;
@@ -164,17 +174,18 @@ __global__ void __launch_bounds__(512)
   for (int i = 0; i < kSteps; ++i) {
     const int b = bks[i];
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
-    if (b >= 0 && lane == __ffs(peers) - 1) mybase[b] += __popc(peers);
+    if (b >= 0 && lane == __ffs(peers) - 1) mycnt[b] = (uint16_t)(mycnt[b] + __popc(peers));
     __syncwarp();
   }
   __syncthreads();
-  // 2) exclusive scan over warps, seeded with the tile's offset for the bucket
+  // 2) the tile's offset per bucket, and an exclusive scan over the warps
   const int32_t* h = hist + (int64_t)seg * nb * tiles + tl;
   for (int b = threadIdx.x; b < nb; b += blockDim.x) {
-    int32_t run = h[(int64_t)b * tiles];
+    toff[b] = h[(int64_t)b * tiles];
+    uint32_t run = 0;
     for (int w = 0; w < nw; ++w) {
-      const int32_t c = base[w * nb + b];
-      base[w * nb + b] = run;
+      const uint32_t c = cnt[w * nb + b];
+      cnt[w * nb + b] = (uint16_t)run;
       run += c;
     }
   }
@@ -187,9 +198,9 @@ __global__ void __launch_bounds__(512)
     const int b = bks[i];
     const uint32_t peers = __match_any_sync(0xffffffffu, b);
     int slot = 0;
-    if (b >= 0) slot = mybase[b] + __popc(peers & lanemask_lt());
+    if (b >= 0) slot = toff[b] + mycnt[b] + __popc(peers & lanemask_lt());
     __syncwarp();
-    if (b >= 0 && lane == __ffs(peers) - 1) mybase[b] += __popc(peers);
+    if (b >= 0 && lane == __ffs(peers) - 1) mycnt[b] = (uint16_t)(mycnt[b] + __popc(peers));
     __syncwarp();
     if (b >= 0) {
       perm[so + slot] = t;

@@ -110,6 +110,15 @@ def test_calls_reject_bad_arguments_before_launch(lib):
     assert lib.lsh_attn_workspace_size(None, ctypes.byref(ctypes.c_size_t())) == 1
 
 
+def test_wait_selftest_rejects_bad_arguments_before_launch(lib):
+    f = lib.lsh_attn_selftest_wait_timeout
+    p, z = ctypes.c_void_p(4096), None
+    assert f(z, 4096, 1000, z) == 1          # no workspace
+    assert f(p, 16, 1000, z) == 1            # smaller than the status header
+    assert f(p, 4096, 0, z) == 1             # limit out of range
+    assert f(p, 4096, 2000001, z) == 1
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert lib.lsh_attn_status_string(s).startswith(b"LSH_")
