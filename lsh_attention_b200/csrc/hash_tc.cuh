@@ -123,7 +123,8 @@ template <int D>
 __global__ void __launch_bounds__(128)
     k_hash_refine(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Rt,
                   const uint64_t* __restrict__ queue, int64_t cap, int32_t* __restrict__ buckets,
-                  int n, int nb, int rounds, int rows_per_round, const WsHeader* __restrict__ hdr) {
+                  int n, int nb, int rounds, int rows_per_round, const WsHeader* __restrict__ hdr,
+                  int32_t* __restrict__ hist, int sort_tile, int sort_tiles) {
   constexpr int E = kRefineBatch;
   __shared__ double xs[E][D];
   __shared__ double wv[4][E];
@@ -161,11 +162,18 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[c][e] = 0.0;
       }
+      // the next 8 k of every column are loaded while these are summed
+      uint4 nxt[C];
+#pragma unroll
+      for (int c = 0; c < C; ++c) nxt[c] = __ldg(rr[c]);
 #pragma unroll 1
       for (int k8 = 0; k8 < D / 8; ++k8) {
         float f[C][8];
 #pragma unroll
-        for (int c = 0; c < C; ++c) Vec16<__nv_bfloat16>::unpack(__ldg(rr[c] + k8), f[c]);
+        for (int c = 0; c < C; ++c) {
+          Vec16<__nv_bfloat16>::unpack(nxt[c], f[c]);
+          if (k8 + 1 < D / 8) nxt[c] = __ldg(rr[c] + k8 + 1);
+        }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           double xv[E];
@@ -212,7 +220,16 @@ __global__ void __launch_bounds__(128)
       const int64_t row = (int64_t)qr[e0 + tid];
       const int64_t bh = row / n;
       const int t = (int)(row % n);
-      buckets[(bh * rounds + r) * n + t] = b;
+      int32_t* slot = buckets + (bh * rounds + r) * n + t;
+      if (hist != nullptr) {  // move the count of a token whose bucket changed
+        const int old = *slot;
+        if (old != b) {
+          int32_t* hs = hist + (bh * rounds + r) * (int64_t)nb * sort_tiles + t / sort_tile;
+          atomicAdd(hs + (int64_t)old * sort_tiles, -1);
+          atomicAdd(hs + (int64_t)b * sort_tiles, 1);
+        }
+      }
+      *slot = b;
     }
     __syncthreads();
   }
@@ -224,7 +241,9 @@ struct HashTcArgs {
   uint64_t* refine;   // near-tie queues, one of `cap` entries per round
   int64_t cap;        // BH * n
   WsHeader* hdr;      // rnorm bits in hdr->pad[0, 16), queue lengths in hdr->pad[16, 32)
+  int32_t* hist;      // the sort's [seg][nb][sort_tiles] counts (zeroed), or null
   int n, nb, rounds, tiles_per_seq, tiles, ctas_per_group;
+  int sort_tile, sort_tiles;  // tokens per sort tile, sort tiles per sequence
 };
 
 // Running top-2 of |p| with the argmax and its signed value.
@@ -548,6 +567,10 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
             const int bucket = idx + (sv < 0.f ? p.half : 0);
             const int64_t at = ((int64_t)bh * a.rounds + r) * a.n + t;
             a.buckets[at] = bucket;
+            if (a.hist != nullptr)  // the sort's tile histogram, counted here
+              atomicAdd(a.hist + ((int64_t)(bh * a.rounds + r) * a.nb + bucket) * a.sort_tiles +
+                            t / a.sort_tile,
+                        1);
             if (!(m1 - m2 > tau)) {
               atomicAdd(&a.hdr->hash_refined, 1u);
               const uint32_t k = atomicAdd(&a.hdr->pad[16 + r], 1u);

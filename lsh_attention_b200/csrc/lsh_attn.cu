@@ -165,10 +165,14 @@ lsh_status launch_hash_exact(const Dims& D, const void* x, const void* R, int32_
 }
 
 // bf16: tcgen05 projection + top-2 screen, fp64 re-decision of near ties.
+// hist: when not null, the sort's tile histograms are counted by the hash
+// (and *hist_done set); otherwise the sort counts them itself.
 lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const void* R,
-                          int32_t* buckets, void* ws, cudaStream_t st, void* const* ev) {
+                          int32_t* buckets, void* ws, cudaStream_t st, void* const* ev,
+                          int32_t* hist = nullptr, bool* hist_done = nullptr) {
   const HashTcPlan p = hash_tc_plan(D.d, D.nb, D.rounds);
   lsh_status s;
+  if (hist_done) *hist_done = false;
   if (p.group == 0) {
     if ((s = mark(ev, 1, st)) != LSH_OK) return s;
     if ((s = launch_hash_exact(D, x, R, buckets, st, true)) != LSH_OK) return s;
@@ -198,6 +202,12 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
   a.rounds = D.rounds;
   a.tiles_per_seq = (D.n + kHashTile - 1) / kHashTile;
   a.tiles = (int)(D.BH * a.tiles_per_seq);
+  a.hist = hist;
+  a.sort_tile = sort_tile(D.nb);
+  a.sort_tiles = D.tiles;
+  if (hist != nullptr &&
+      cudaMemsetAsync(hist, 0, sizeof(int32_t) * (size_t)D.S * D.nb * D.tiles, st) != cudaSuccess)
+    return LSH_ERR_CUDA;
   const int sms = sm_count();
   int per = sms / p.groups;
   if (per < 1) per = 1;
@@ -218,21 +228,27 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
     kern<<<grid, kHashWarps * 32, p.smem, st>>>(tmx, tmr, a, p);
   }
   if ((s = mark(ev, 2, st)) != LSH_OK) return s;
-  dim3 rg((unsigned)((4 * sms + D.rounds - 1) / D.rounds), D.rounds);
+  // eight CTAs per SM over the rounds: a round's queue (a fraction of a percent
+  // of its tokens) is one wave of 8-token batches; surplus CTAs exit at once
+  dim3 rg((unsigned)((8 * sms + D.rounds - 1) / D.rounds), D.rounds);
   if (D.d == 64)
     k_hash_refine<64><<<rg, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine, a.cap,
-                                          buckets, D.n, D.nb, D.rounds, rows_per_round, hdr);
+                                          buckets, D.n, D.nb, D.rounds, rows_per_round, hdr, hist,
+                                          a.sort_tile, a.sort_tiles);
   else
     k_hash_refine<128><<<rg, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), rt, refine,
                                            a.cap, buckets, D.n, D.nb, D.rounds, rows_per_round,
-                                           hdr);
+                                           hdr, hist, a.sort_tile, a.sort_tiles);
   if ((s = last_cuda()) != LSH_OK) return s;
+  if (hist_done) *hist_done = hist != nullptr;
   return mark(ev, 3, st);
 }
 
 lsh_status launch_hash(const Dims& D, const Layout& L, const void* x, const void* R,
-                       int32_t* buckets, void* ws, cudaStream_t st, void* const* ev = nullptr) {
-  if (D.dtype == LSH_BF16) return launch_hash_tc(D, L, x, R, buckets, ws, st, ev);
+                       int32_t* buckets, void* ws, cudaStream_t st, void* const* ev = nullptr,
+                       int32_t* hist = nullptr, bool* hist_done = nullptr) {
+  if (D.dtype == LSH_BF16) return launch_hash_tc(D, L, x, R, buckets, ws, st, ev, hist, hist_done);
+  if (hist_done) *hist_done = false;
   lsh_status s;
   if ((s = mark(ev, 1, st)) != LSH_OK) return s;
   if ((s = launch_hash_exact(D, x, R, buckets, st, false)) != LSH_OK) return s;
@@ -243,12 +259,14 @@ lsh_status launch_hash(const Dims& D, const Layout& L, const void* x, const void
 template <typename T>
 lsh_status launch_sort(const Dims& D, const int32_t* buckets, const void* x, const void* v,
                        int32_t* perm, int32_t* inv, void* xs, void* vs, float* invnorm,
-                       int32_t* hist, WsHeader* hdr, cudaStream_t st, void* const* ev = nullptr) {
+                       int32_t* hist, WsHeader* hdr, cudaStream_t st, void* const* ev = nullptr,
+                       bool hist_ready = false) {
   lsh_status s;
   const int tile = sort_tile(D.nb);
   dim3 grid(D.tiles, (unsigned)D.S);
-  k_sort_hist<<<grid, 256, sizeof(int32_t) * D.nb, st>>>(buckets, D.n, D.nb, tile, D.tiles, hist,
-                                                         hdr);
+  if (!hist_ready)  // else the hash has counted them
+    k_sort_hist<<<grid, 256, sizeof(int32_t) * D.nb, st>>>(buckets, D.n, D.nb, tile, D.tiles,
+                                                           hist, hdr);
   if ((s = mark(ev, 4, st)) != LSH_OK) return s;
   k_sort_scan<<<(unsigned)D.S, 1024, 0, st>>>(hist, D.nb * D.tiles);
   if ((s = mark(ev, 5, st)) != LSH_OK) return s;
@@ -366,9 +384,12 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
   WsHeader* hdr = at<WsHeader>(ws, L.header);
   lsh_status s;
   if ((s = mark(ev, 0, st)) != LSH_OK) return s;
+  bool hist_ready = false;
   if (!buckets) {
     int32_t* bk = at<int32_t>(ws, L.buckets);
-    if ((s = launch_hash(D, L, x, R, bk, ws, st, ev)) != LSH_OK) return s;
+    if ((s = launch_hash(D, L, x, R, bk, ws, st, ev, at<int32_t>(ws, L.hist), &hist_ready)) !=
+        LSH_OK)
+      return s;
     buckets = bk;
   } else {
     for (int i = 1; i <= 3; ++i)
@@ -381,7 +402,7 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
   void* vs = at<unsigned char>(ws, L.vs);
   T* out_r = at<T>(ws, L.out_s);  // each round's output rows, slot order
   if ((s = launch_sort<T>(D, buckets, x, v, perm, inv, xs, vs, invnorm, at<int32_t>(ws, L.hist),
-                          hdr, st, ev)) != LSH_OK)
+                          hdr, st, ev, hist_ready)) != LSH_OK)
     return s;
   if (attn_tc_supported(D))
     s = launch_attn_tc(D, xs, vs, perm, invnorm, out_r, lse, hdr, st);
