@@ -77,6 +77,8 @@ def parse_args():
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default=I.LONG_64K.name, choices=sorted(I.WORKLOADS))
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--ref-seconds", type=float, default=120.0,
+                   help="reference arm: seconds that warm-up plus timed steps should take")
     return p.parse_args()
 
 
@@ -220,7 +222,7 @@ def run_reference(args, w):
     C fp64 oracle (hash, sort, chunk attention, merge) on `hs` heads x `rs`
     rounds of batch 0 over the first `n_s` positions, one OpenMP thread per
     (head, round) unit; n_s is calibrated so warm-up plus steps take about two
-    minutes. Tokens are counted pro rata: B*n * (n_s/n) * (hs/H) * (rs/R)."""
+    minutes (--ref-seconds). Tokens are counted pro rata: B*n * (n_s/n) * (hs/H) * (rs/R)."""
     world, rank, _ = dist_setup("gloo")
     if rank != 0:
         return
@@ -240,7 +242,7 @@ def run_reference(args, w):
         oracle.forward(xs, vs, R[:rs], m, w.causal, nthreads=hs * rs)
         return time.perf_counter() - t0
 
-    budget = 120.0 / max(1, args.steps + args.warmup)  # seconds per step
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)  # seconds per step
     n_s = min(w.n, 4096)
     t0 = step(n_s)  # calibration
     n_s = int(min(w.n, max(m, (n_s * budget / max(t0, 1e-3)) // m * m)))
