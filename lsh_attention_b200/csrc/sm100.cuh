@@ -85,14 +85,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
       "r"(smem_u32(src)), "r"(c0), "r"(c1)
       : "memory");
 }
-// Untiled bulk copy shared -> global (16-byte aligned, size a multiple of 16),
-// bulk-group completion.
-__device__ __forceinline__ void bulk_copy_s2g(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(smem_u32(src)), "r"(bytes)
-               : "memory");
-}
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -185,23 +177,6 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[4][16]) {
       :
       : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[3][16]) {
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(a[0][0]), "+r"(a[0][1]), "+r"(a[0][2]), "+r"(a[0][3]), "+r"(a[0][4]),
-        "+r"(a[0][5]), "+r"(a[0][6]), "+r"(a[0][7]), "+r"(a[0][8]), "+r"(a[0][9]),
-        "+r"(a[0][10]), "+r"(a[0][11]), "+r"(a[0][12]), "+r"(a[0][13]), "+r"(a[0][14]),
-        "+r"(a[0][15]), "+r"(a[1][0]), "+r"(a[1][1]), "+r"(a[1][2]), "+r"(a[1][3]),
-        "+r"(a[1][4]), "+r"(a[1][5]), "+r"(a[1][6]), "+r"(a[1][7]), "+r"(a[1][8]),
-        "+r"(a[1][9]), "+r"(a[1][10]), "+r"(a[1][11]), "+r"(a[1][12]), "+r"(a[1][13]),
-        "+r"(a[1][14]), "+r"(a[1][15]), "+r"(a[2][0]), "+r"(a[2][1]), "+r"(a[2][2]),
-        "+r"(a[2][3]), "+r"(a[2][4]), "+r"(a[2][5]), "+r"(a[2][6]), "+r"(a[2][7]),
-        "+r"(a[2][8]), "+r"(a[2][9]), "+r"(a[2][10]), "+r"(a[2][11]), "+r"(a[2][12]),
-        "+r"(a[2][13]), "+r"(a[2][14]), "+r"(a[2][15])
-      :
-      : "memory");
-}
-
 // Untiled bulk copy global -> shared (16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
                                               uint64_t* bar) {
