@@ -218,6 +218,9 @@ EDGE = [
     ("max-buckets", 1, 1, 8192, 64, 4096, 64, 1, True, "bf16"),
     ("noncausal-bf16-d128", 1, 2, 1024, 128, 32, 64, 2, False, "bf16"),
     ("noncausal-bf16-d64", 2, 1, 640, 64, 16, 64, 3, False, "bf16"),
+    # more rounds than a merge lane group of bf16 d64 has lanes (8), and the most rounds
+    ("many-rounds-bf16-d64", 1, 2, 512, 64, 16, 64, 12, True, "bf16"),
+    ("max-rounds-bf16-d128", 1, 1, 512, 128, 16, 64, 16, True, "bf16"),
 ]
 
 
