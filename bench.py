@@ -49,6 +49,7 @@ STAGE_KERNEL = {"hash": "hash_mma", "sort_gather": "row_gather",
 # DRAM bytes (read + write) per launch from one ncu capture of the long-64k
 # workload, valid only while the kernel's source file is unchanged (sha256
 # of the file at capture time); see profiles/.
+NCU_WORKLOAD = I.LONG_64K.name
 NCU_TRAFFIC = {
     "hash_prep": {"bytes": 532000, "file": "hash_tc.cuh",
         "sha256": "982d14f4a39e9dac2c63b2033077b2dd222f68c734c9a191ea6ea366ce10e356"},
@@ -62,8 +63,8 @@ NCU_TRAFFIC = {
         "sha256": "e031792086f8fef697f441014adf16e9a9b36d922f1a623610bc2e5e46c4b5ab"},
     "row_gather": {"bytes": 1513671000, "file": "gather.cuh",
         "sha256": "e6ed6996ab9b55d7b4ab341085d7fa0a4c9c38b1532727b5bb8fad26bde2238a"},
-    "chunk_attention": {"bytes": 1652110000, "file": "attn_tc.cuh",
-        "sha256": "662aea74507cfaa09642c7e3d073502e380987346a7690e33e3af2093889c234"},
+    "chunk_attention": {"bytes": 1653029952, "file": "attn_tc.cuh",
+        "sha256": "1e52dd753ec04f9e2910d0c668cd8317e16cf5d6e703df6a8962d1d8303d387f"},
     "unsort_merge": {"bytes": 672942000, "file": "merge.cuh",
         "sha256": "f313dd4622da3353060cb7b84324a099bfef2be35a4e693135b8674f34cd17db"},
 }
@@ -388,7 +389,7 @@ def run_ours(args, w):
                 "peak": pk["hbm_gbs"]}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     roof["kernel"] = dom
-    roof["traffic"] = traffic_of(dom)
+    roof["traffic"] = traffic_of(dom, w.name)
     roof["peak_source"] = "of measured (MEASURED_PEAKS.json)" if pk_kind == "measured" else \
         "of fallback"
     line = {
@@ -416,11 +417,12 @@ def launches_per_forward(buckets_given: bool) -> int:
     return (4 if buckets_given else 3 + 3) + 1 + 1
 
 
-def traffic_of(kernel: str):
-    """ncu DRAM bytes per launch of `kernel`, if its source is unchanged."""
+def traffic_of(kernel: str, workload: str):
+    """ncu DRAM bytes per launch of `kernel`, if the capture was of this
+    workload and the kernel's source is unchanged since."""
     import hashlib
     rec = NCU_TRAFFIC.get(kernel)
-    if rec is None:
+    if rec is None or workload != NCU_WORKLOAD:
         return None
     path = os.path.join(ROOT, "lsh_attention_b200", "csrc", rec["file"])
     with open(path, "rb") as f:

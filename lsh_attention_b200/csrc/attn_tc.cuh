@@ -266,29 +266,39 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         if (bound > kAttnBoundMax) bound = mx == -INFINITY ? 0.f : mx;
       }
       float sum0 = 0.f, sum1 = 0.f;
+      // 32-key batches per TMEM wait: two at d = 64, where the softmax paces
+      // the pipeline (more exponents in flight), one at d = 128, where the
+      // registers are spoken for
+      constexpr int BPW = D == 64 ? 2 : 1;
 #pragma unroll 1
-      for (int b = 0; b < 4; ++b) {
-        uint32_t v[32];
-        tmem_ld32(ts + wcol + b * 32, v);
-        tmem_wait_ld();
-        uint32_t pk[16];
-        const float4* kt4 = reinterpret_cast<const float4*>(kt + wcol + b * 32);
+      for (int b2 = 0; b2 < 4; b2 += BPW) {
+        uint32_t v[BPW][32];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float4 t = kt4[c >> 1];  // (scale, position) of keys c and c + 1
-          // every exponent is computed, then invisible keys are masked: no
-          // divergent branch per key
-          const float e0 = ex2_approx(fmaf(__uint_as_float(v[c]), t.x, -bound));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(v[c + 1]), t.z, -bound));
-          const float p0 = visible(__float_as_int(t.y)) ? e0 : 0.f;
-          const float p1 = visible(__float_as_int(t.w)) ? e1 : 0.f;
-          sum0 += p0;
-          sum1 += p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
+        for (int h = 0; h < BPW; ++h) tmem_ld32(ts + wcol + (b2 + h) * 32, v[h]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < BPW; ++h) {
+          const int b = b2 + h;
+          uint32_t pk[16];
+          const float4* kt4 = reinterpret_cast<const float4*>(kt + wcol + b * 32);
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float4 t = kt4[c >> 1];  // (scale, position) of keys c and c + 1
+            // every exponent is computed, then invisible keys are masked: no
+            // divergent branch per key
+            const float e0 = ex2_approx(fmaf(__uint_as_float(v[h][c]), t.x, -bound));
+            const float e1 = ex2_approx(fmaf(__uint_as_float(v[h][c + 1]), t.z, -bound));
+            const float p0 = visible(__float_as_int(t.y)) ? e0 : 0.f;
+            const float p1 = visible(__float_as_int(t.w)) ? e1 : 0.f;
+            sum0 += p0;
+            sum1 += p1;
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          // P column c holds keys 2c, 2c+1: batch b lands in columns
+          // [wcol/2 + 16b, wcol/2 + 16b + 16), S columns already read (or,
+          // for wcol = 64 and b < 2, columns outside this row's window)
+          tmem_st16(ts + wcol / 2 + b * 16, pk);
         }
-        // P column c holds keys 2c, 2c+1: chunk b lands in columns
-        // [wcol/2 + 16b, wcol/2 + 16b + 16), behind every S column still unread
-        tmem_st16(ts + wcol / 2 + b * 16, pk);
       }
       uint32_t z[16];
 #pragma unroll
