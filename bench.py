@@ -52,19 +52,19 @@ STAGE_KERNEL = {"hash": "hash_mma", "sort_gather": "row_gather",
 NCU_WORKLOAD = I.LONG_64K.name
 NCU_TRAFFIC = {
     "hash_prep": {"bytes": 532000, "file": "hash_tc.cuh",
-        "sha256": "982d14f4a39e9dac2c63b2033077b2dd222f68c734c9a191ea6ea366ce10e356"},
-    "hash_mma": {"bytes": 150564000, "file": "hash_tc.cuh",
-        "sha256": "982d14f4a39e9dac2c63b2033077b2dd222f68c734c9a191ea6ea366ce10e356"},
+        "sha256": "37f57d7a8e89a1eeafa3c2e622f96c5a6d2ad920cdf54cb8c39cddab6f44948e"},
+    "hash_mma": {"bytes": 150716200, "file": "hash_tc.cuh",
+        "sha256": "37f57d7a8e89a1eeafa3c2e622f96c5a6d2ad920cdf54cb8c39cddab6f44948e"},
     "hash_refine": {"bytes": 2748000, "file": "hash_tc.cuh",
-        "sha256": "982d14f4a39e9dac2c63b2033077b2dd222f68c734c9a191ea6ea366ce10e356"},
+        "sha256": "37f57d7a8e89a1eeafa3c2e622f96c5a6d2ad920cdf54cb8c39cddab6f44948e"},
     "sort_scan": {"bytes": 4204000, "file": "sort.cuh",
         "sha256": "e031792086f8fef697f441014adf16e9a9b36d922f1a623610bc2e5e46c4b5ab"},
     "sort_rank": {"bytes": 12598000, "file": "sort.cuh",
         "sha256": "e031792086f8fef697f441014adf16e9a9b36d922f1a623610bc2e5e46c4b5ab"},
     "row_gather": {"bytes": 1513671000, "file": "gather.cuh",
         "sha256": "e6ed6996ab9b55d7b4ab341085d7fa0a4c9c38b1532727b5bb8fad26bde2238a"},
-    "chunk_attention": {"bytes": 1653029952, "file": "attn_tc.cuh",
-        "sha256": "1e52dd753ec04f9e2910d0c668cd8317e16cf5d6e703df6a8962d1d8303d387f"},
+    "chunk_attention": {"bytes": 1656132536, "file": "attn_tc.cuh",
+        "sha256": "ef34b0f22a208e36832902dd14b8d51dc86fdddd67df14426033343ba0d3c0df"},
     "unsort_merge": {"bytes": 672942000, "file": "merge.cuh",
         "sha256": "f313dd4622da3353060cb7b84324a099bfef2be35a4e693135b8674f34cd17db"},
 }

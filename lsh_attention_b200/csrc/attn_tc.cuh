@@ -224,7 +224,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     const float c_scale = kLog2e / sqrtf((float)D);
     for (int i = 0; i < nu; ++i) {
       const int s = i & 1, k = i >> 1;
-      if (!mbar_wait(sfull + s, k & 1)) { fail(); break; }
+      const bool got = mbar_wait(sfull + s, k & 1);
+      if (!got) fail();
       tc_fence_after();
       const int64_t seg = unit_seg(i);
       const int c0 = unit_c0(i);
@@ -232,14 +233,16 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       // per-key table: logit scale (log2 units) and position; keys outside
       // [0, n) get a position that every query's test rejects
       float2* kt = ktab + s * kAttnKeys;
-      for (int j = st; j < kAttnKeys; j += 128) {
+      for (int j = st; got && j < kAttnKeys; j += 128) {
         const int ks = k0 + j;
         const bool valid = ks >= 0 && ks < a.n;
         kt[j] = make_float2(valid ? kinv[s * kAttnKeys + j] * c_scale : 0.f,
                             __int_as_float(valid ? kpos[s * kAttnKeys + j] : kNoKey));
       }
       const float qinv = kinv[s * kAttnKeys + kAttnM + row];
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // the four softmax warps
+      // the four softmax warps; a failure seen by any of them stops all four
+      // here, so none is left waiting at this barrier
+      if (bar_sync_any(1, 128, !got || *abort_flag)) break;
       if (lane == 0) mbar_arrive(xfree + s);  // metadata of this stage consumed
       const int qpos = __float_as_int(kt[kAttnM + row].y);
       // stabiliser: ||q|| log2(e) / sqrt(d) bounds every logit of the row

@@ -475,8 +475,8 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
       const int xb = it & 1, xk = it >> 1;
       const int bh = tile / a.tiles_per_seq;
       const int t = (tile % a.tiles_per_seq) * kHashTile + row;
-      // Failures set abort_flag before the next named barrier, so both warps
-      // of a quadrant leave the loop after the same barrier.
+      // A failure anywhere sets abort_flag; the quadrant's warps OR it at
+      // their combine barrier and leave the loop together after it.
       bool ok = true;
       // ||x_row||^2 in parts: warp h >= 1 sums the row's 16-byte chunks
       // cc = h - 1 (mod PO) from the swizzled tile (chunk c of a 128-byte
@@ -547,8 +547,9 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
           slot[(h - 1) * 32] = make_float4(m1, m2, __int_as_float(idx), sv);
           sslot[(h - 1) * 32] = ss;
         }
-        asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(32 * kHashEpiPerQuad) : "memory");
-        stop = *abort_flag != 0;
+        // the quadrant's warps decide together whether to stop (a failure
+        // anywhere sets abort_flag), so they leave after the same barrier
+        stop = bar_sync_any(1 + q, 32 * kHashEpiPerQuad, *abort_flag != 0);
         if (stop) break;
         if (h == 0) {
 #pragma unroll

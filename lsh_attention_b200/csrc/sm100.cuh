@@ -64,6 +64,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return true;
 }
 
+// Named barrier `id` over `count` threads that also ORs a flag across them:
+// every participant gets the same answer, so a decision to stop is taken by
+// all of them at the same barrier.
+__device__ __forceinline__ bool bar_sync_any(int id, int count, bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pc, pr;\n\t"
+      "setp.ne.u32 pc, %1, 0;\n\t"
+      "bar.red.or.pred pr, %2, %3, pc;\n\t"
+      "selp.u32 %0, 1, 0, pr;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)flag), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 // ---------------------------------------------------------------- TMA
 // 2D tiled load into shared memory, completion counted on `bar`.
 // c0 is the innermost coordinate (elements), c1 the row.
