@@ -7,6 +7,8 @@ never do. It shares no code with the CUDA path.
 The arithmetic lives in ``lsh_oracle.c`` (plain C99, fp64, OpenMP over
 independent (batch, head, round) units). This module builds it with gcc if the
 shared object is missing and marshals numpy / torch arrays into fp64.
+``backward.py`` restates the forward in float64 torch operations and gives its
+gradients with respect to x and v (for a backward pass to be checked against).
 
 Every input is widened to fp64 exactly (fp32 and bf16 values are fp64 values),
 so the oracle evaluates the definition on the very numbers the GPU consumes.
