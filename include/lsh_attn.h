@@ -176,12 +176,18 @@ lsh_status lsh_attn_selftest_wait_timeout(void *workspace, size_t workspace_byte
  *     4*B*H*Rn*n bytes of scratch, T = 256 * clamp(8192 / nb, 1, 8); larger
  *     problems return LSH_ERR_UNSUPPORTED and write nothing (use lsh_attn_sort).
  *   - The first call on a device looks up the scratch's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *     that device current) and caches it for the life of the process; make
+ *     that first call before any stream capture. cudaDeviceReset on a device
+ *     makes the cached address stale: after a reset, do not call this entry
+ *     point on that device again in the same process.
  *   - Every call on a device shares the one scratch, whose contents persist
  *     from the previous call: calls that may overlap on the GPU (different
  *     streams without ordering between them) race and must not be issued.
- *   - Errors as for lsh_attn_sort; kernel-side status is not readable here. */
+ *   - Host-side errors as for lsh_attn_sort. The kernels' status word lives
+ *     in the shared scratch and no call reads it, so bucket ids outside
+ *     [0, nb) are clamped into range SILENTLY here (the perm is that of the
+ *     clamped ids and the call returns LSH_OK); lsh_attn_sort reports the
+ *     same input as LSH_ERR_DEVICE. */
 lsh_status lsh_attn_sort_noalloc(const lsh_attn_desc *desc, const int32_t *buckets,
                                  int32_t *perm, void *stream);
 

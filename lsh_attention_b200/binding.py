@@ -105,6 +105,23 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _on_current_device(stream=None, **tensors) -> None:
+    """The library launches on the current CUDA device and dereferences every
+    pointer there: raise ValueError, before anything is launched, unless every
+    given tensor (and the stream, if one is given) lives on that device."""
+    cur = torch.cuda.current_device()
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.device.index != cur:
+            raise ValueError(f"{name} is on {t.device}, but the current device is cuda:{cur}; "
+                             f"call inside `with torch.cuda.device({t.device})`")
+    if stream is not None and stream.device.index != cur:
+        raise ValueError(f"stream is on {stream.device}, but the current device is cuda:{cur}")
+
+
 def _require(t: torch.Tensor, name: str, dtype, shape) -> None:
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -142,6 +159,7 @@ def workspace(desc: LshAttnDesc, device, stream=None) -> torch.Tensor:
 
 def lsh_attn_hash(x, R, n_buckets: int, buckets=None, ws=None, stream=None):
     """Bucket ids [B, H, rounds, n] int32 of x [B, H, n, d] under R [rounds, d, nb/2]."""
+    _on_current_device(stream, x=x, R=R, buckets=buckets, ws=ws)
     B, H, n, d = x.shape
     rounds = R.shape[0]
     _require(x, "x", None, None)
@@ -162,6 +180,7 @@ def lsh_attn_sort(buckets, n_buckets: int, x=None, v=None, perm=None, xs=None, v
     """Stable sort by (bucket, position) of every (batch, head, round).
     Returns perm [B, H, rounds, n] int32, and (xs, vs) sorted row copies when
     x and v are given."""
+    _on_current_device(stream, buckets=buckets, x=x, v=v, perm=perm, xs=xs, vs=vs, ws=ws)
     B, H, rounds, n = buckets.shape
     _require(buckets, "buckets", torch.int32, None)
     if x is not None:
@@ -193,6 +212,7 @@ def lsh_attn_forward(x, v, R=None, *, n_buckets: int, chunk: int, causal: bool, 
     [B, H, rounds, n] fp32). `events`: PROFILE_EVENTS recorded
     torch.cuda.Event objects marking the kernel boundaries
     (lsh_attn_forward_profiled)."""
+    _on_current_device(stream, x=x, v=v, R=R, buckets=buckets, out=out, lse=lse, ws=ws)
     B, H, n, d = x.shape
     _require(x, "x", None, None)
     _require(v, "v", x.dtype, tuple(x.shape))
@@ -228,6 +248,7 @@ def lsh_attn_forward(x, v, R=None, *, n_buckets: int, chunk: int, causal: bool, 
 def lsh_attn_sort_noalloc(buckets, n_buckets: int, perm=None, stream=None):
     """perm [B, H, rounds, n] of the stable bucket sort without any workspace:
     the library's fixed device scratch is used (see lsh_attn.h)."""
+    _on_current_device(stream, buckets=buckets, perm=perm)
     B, H, rounds, n = buckets.shape
     _require(buckets, "buckets", torch.int32, None)
     desc = make_desc(B, H, n, 64, n_buckets, 1, rounds, False, torch.bfloat16)
@@ -240,6 +261,7 @@ def lsh_attn_sort_noalloc(buckets, n_buckets: int, perm=None, stream=None):
 
 
 def lsh_attn_get_diag(ws, stream=None) -> dict:
+    _on_current_device(stream, ws=ws)
     d = LshAttnDiag()
     _check(load().lsh_attn_get_diag(_ptr(ws), _stream(stream), ctypes.byref(d)))
     return {"status": d.status, "hash_refined": d.hash_refined,
@@ -247,6 +269,7 @@ def lsh_attn_get_diag(ws, stream=None) -> dict:
 
 
 def lsh_attn_get_device_status(ws, stream=None) -> int:
+    _on_current_device(stream, ws=ws)
     return load().lsh_attn_get_device_status(_ptr(ws), _stream(stream))
 
 
@@ -255,5 +278,6 @@ def lsh_attn_selftest_wait_timeout(ws, limit_us: int, stream=None) -> None:
     least 256 bytes): a wait that nothing completes gives up after
     `limit_us` and records LSH_ERR_TIMEOUT (read it with
     lsh_attn_get_device_status)."""
+    _on_current_device(stream, ws=ws)
     _check(load().lsh_attn_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(),
                                                  int(limit_us), _stream(stream)))

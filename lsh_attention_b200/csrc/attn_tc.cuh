@@ -105,6 +105,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   uint64_t* statf = bars + 16;   // [4] row sums written (4 softmax warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
+  uint64_t* drain = bars + 22;   // MMA issuer: every issued MMA has completed
+  volatile int* drain_fail = reinterpret_cast<volatile int*>(bars + 23);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t u0 = blockIdx.x * a.pairs_per_cta;
@@ -125,7 +127,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     mbar_init(ofull, 1);
     mbar_init(ofree, 4);
     for (int i = 0; i < kAttnStats; ++i) mbar_init(statf + i, 4);
+    mbar_init(drain, 1);
     *abort_flag = 0;
+    *drain_fail = 0;
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
@@ -148,6 +152,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       prefetch_tensormap(&tmx);
       prefetch_tensormap(&tmv);
       bool ok = true;
+      int lastx[2] = {-1, -1}, lastv[2] = {-1, -1};  // last phase issued per stage
       for (int i = 0; ok && i < nu && !*abort_flag; ++i) {
         const int s = i & 1, k = i >> 1;
         const int64_t seg = unit_seg(i);
@@ -163,12 +168,20 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
                       xfull + s);
         bulk_copy_g2s(kpos + s * kAttnKeys + (lo - k0), a.perm + seg * a.n + lo, mbytes,
                       xfull + s);
+        lastx[s] = k;
         if (k > 0 && !mbar_wait(vfree + s, (k - 1) & 1)) { ok = false; break; }
         mbar_expect_tx(vfull + s, TILE);
         for (int kh = 0; kh < KH; ++kh)
           tma_load_2d(vt + s * TILE + kh * BOX, &tmv, vfull + s, kh * 64, row);
+        lastv[s] = k;
       }
       if (!ok) fail();
+      // No copy may still be writing this CTA's shared memory when it exits:
+      // wait (bounded) for the last phase issued on every stage.
+      for (int s = 0; s < 2; ++s)
+        if ((lastx[s] >= 0 && !mbar_wait(xfull + s, lastx[s] & 1)) ||
+            (lastv[s] >= 0 && !mbar_wait(vfull + s, lastv[s] & 1)))
+          *drain_fail = 1;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -213,6 +226,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       for (int i = 0; ok && i < nu && !*abort_flag; ++i)
         ok = (i + 1 >= nu || issue_s(i + 1)) && issue_pv(i);
       if (!ok) fail();
+      // TMEM is freed below: every MMA issued must have completed first
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0)) *drain_fail = 1;
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ softmax
@@ -383,7 +399,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  // after a drain that gave up, TMEM is left allocated rather than freed
+  // under a running MMA; the status word already records the timeout
+  if (warp == 1 && !*drain_fail) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

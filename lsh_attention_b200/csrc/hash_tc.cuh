@@ -355,6 +355,8 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
   uint64_t* acc_empty = bars + 7;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
+  uint64_t* drain = bars + 11;  // MMA issuer: every issued MMA has completed
+  volatile int* drain_fail = reinterpret_cast<volatile int*>(bars + 12);
   constexpr int PO = kHashEpiPerQuad - 1;  // warps of a quadrant that report to h = 0
   float4* comb = reinterpret_cast<float4*>(bars + 16);  // [2][4][PO][32]
   float* ssb = reinterpret_cast<float*>(comb + 2 * 4 * PO * 32);  // [2][4][PO][32]
@@ -374,7 +376,9 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
       mbar_init(acc_full + i, 1);
       mbar_init(acc_empty + i, 4 * kHashEpiPerQuad);  // every epilogue warp
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
+    *drain_fail = 0;
     fence_mbar_init();
   }
   if (threadIdx.x < a.rounds)  // per-round bound of max_j ||R_j|| (k_hash_prep)
@@ -403,6 +407,7 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
             tma_load_2d(dst, &tmr, r_full, kh * 64, ((r0 + rl) * p.ch + c) * p.nc);
           }
       int it = 0;
+      int lastx[2] = {-1, -1};  // last phase issued per x buffer
       for (int tile = li; tile < a.tiles; tile += a.ctas_per_group, ++it) {
         const int xb = it & 1, xk = it >> 1;
         if (xk > 0 && !mbar_wait(x_empty + xb, (xk - 1) & 1)) { fail(); break; }
@@ -412,7 +417,13 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
         mbar_expect_tx(x_full + xb, KH * XBOX);
         for (int kh = 0; kh < KH; ++kh)
           tma_load_2d(xbuf + (xb * KH + kh) * XBOX, &tmx, x_full + xb, kh * 64, row0);
+        lastx[xb] = xk;
       }
+      // No copy may still be writing this CTA's shared memory when it exits:
+      // wait (bounded) for the rotations and the last phase of each x buffer.
+      if (!mbar_wait(r_full, 0)) *drain_fail = 1;
+      for (int b = 0; b < 2; ++b)
+        if (lastx[b] >= 0 && !mbar_wait(x_full + b, lastx[b] & 1)) *drain_fail = 1;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -462,6 +473,9 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
         }
         mma_commit(x_empty + xb);
       }
+      // TMEM is freed below: every MMA issued must have completed first
+      mma_commit(drain);
+      if (!mbar_wait(drain, 0)) *drain_fail = 1;
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -585,7 +599,9 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  // after a drain that gave up, TMEM is left allocated rather than freed
+  // under a running MMA; the status word already records the timeout
+  if (warp == 1 && !*drain_fail) {
     tc_fence_after();
     tmem_dealloc(tmem, 2 * p.tmem_cols);
   }

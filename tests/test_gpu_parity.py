@@ -57,8 +57,10 @@ def sample_positions(n, k=192, seed=3):
 
 
 SMALL = [I.TINY_F32, I.BF16_SHORT]
+# the n x rounds sweep, isotropic and clustered: 16 points with n <= 8K
+# checked in full, 16 with n >= 32K checked on sampled heads and positions
 SWEEP_SMALL = [w for w in I.sweep_workloads() if w.n <= 8192]
-SWEEP_LARGE = [w for w in I.sweep_workloads() if w.n >= 32768 and w.rounds in (1, 4)]
+SWEEP_LARGE = [w for w in I.sweep_workloads() if w.n >= 32768]
 
 
 # --------------------------------------------------------------------------
@@ -138,7 +140,7 @@ def oracle_buckets(w, x, R):
     return torch.from_numpy(b)
 
 
-@pytest.mark.parametrize("w", SMALL + SWEEP_SMALL[::2], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", SMALL + SWEEP_SMALL, ids=lambda w: w.name)
 def test_forward_full(w):
     """Whole outputs against the oracle, identical buckets on both sides."""
     x, v = I.make_qkv(w)
@@ -155,8 +157,10 @@ def test_forward_full(w):
 
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
 def test_forward_internal_hash(w):
-    """buckets=NULL hashes inside the call: equals the oracle's own full forward
-    (the hash is bit-exact here), and equals the GPU forward fed the GPU hash."""
+    """buckets=NULL hashes inside the call: the GPU's bucket ids must equal the
+    oracle's bit for bit (no near-tie allowance: the bf16 hash re-decides near
+    ties exactly), the output must equal the oracle's own full forward, and
+    the GPU forward fed the GPU hash must give the same bits."""
     x, v = I.make_qkv(w)
     R = I.make_rotations(w)
     xg, vg, Rg = to_gpu(x, v, R)
@@ -164,42 +168,89 @@ def test_forward_internal_hash(w):
                                    causal=w.causal)
     ref_out, ref_lse, ref_bk = oracle.forward(x, v, R, w.chunk, w.causal)
     gbk = lb.lsh_attn_hash(xg, Rg, w.n_buckets)
-    _, margin = oracle.hash_all(x, R)
-    if check_buckets(gbk.cpu().numpy(), ref_bk, margin, w.name) == 0:
-        check_close(out.float().cpu().numpy(), ref_out, w.dtype, f"{w.name} out")
-        check_close(lse.cpu().numpy(), ref_lse, w.dtype, f"{w.name} lse")
+    np.testing.assert_array_equal(gbk.cpu().numpy(), ref_bk)
+    check_close(out.float().cpu().numpy(), ref_out, w.dtype, f"{w.name} out")
+    check_close(lse.cpu().numpy(), ref_lse, w.dtype, f"{w.name} lse")
     out2, lse2 = lb.lsh_attn_forward(xg, vg, None, n_buckets=w.n_buckets, chunk=w.chunk,
                                      causal=w.causal, buckets=gbk)
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
 
 
-@pytest.mark.parametrize("w,heads", [(I.IMAGE_12K, [0, 7]), (I.LONG_64K, [0, 5])] +
+@pytest.mark.parametrize("w,heads", [(I.LONG_64K, [0, 5]), (I.IMAGE_12K, [0, 7])] +
                          [(s, [0, 7]) for s in SWEEP_LARGE],
                          ids=lambda p: p.name if hasattr(p, "name") else str(p))
-def test_forward_sampled(w, heads):
-    """Full-size launch in the bench's configuration; the oracle evaluates sampled
-    positions of sampled heads with the oracle's own buckets for those heads."""
+def test_forward_timed_path(w, heads):
+    """The bench's call at full size: lsh_attn_forward(x, v, R, buckets=NULL),
+    where the tensor-core hash also counts the sort's histograms and the fp64
+    re-decision corrects them.
+      1. On the sampled heads the GPU's bucket ids (every round, every
+         position) equal the oracle's hash bit for bit.
+      2. The timed call's out and lse equal, bit for bit over every head, the
+         GPU forward fed those bucket ids (the separate histogram pass), so the
+         fused histograms give the same permutation.
+      3. At sampled positions of the sampled heads, out and lse match the
+         oracle's forward on the oracle's own ids."""
     x, v = I.make_qkv(w)
     R = I.make_rotations(w)
-    bk = I.make_buckets(w)  # other heads: any valid ids
-    big = w.n * w.n_buckets * w.rounds > 2 ** 27
-    for h in heads:
-        xb = x[:1, h:h + 1] if big else x[:, h:h + 1]
-        b, _ = oracle.hash_all(xb, R)
-        bk[: b.shape[0], h] = torch.from_numpy(b[:, 0])
-    xg, vg, bkg = to_gpu(x, v, bk)
-    out, lse = lb.lsh_attn_forward(xg, vg, None, n_buckets=w.n_buckets, chunk=w.chunk,
-                                   causal=w.causal, buckets=bkg)
+    xg, vg, Rg = to_gpu(x, v, R)
+    kw = dict(n_buckets=w.n_buckets, chunk=w.chunk, causal=w.causal)
+    out, lse = lb.lsh_attn_forward(xg, vg, Rg, **kw)
+    out, lse = out.clone(), lse.clone()
+    gbk = lb.lsh_attn_hash(xg, Rg, w.n_buckets)
+    out2, lse2 = lb.lsh_attn_forward(xg, vg, None, buckets=gbk, **kw)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2), \
+        "the fused-histogram forward differs from the caller-bucket forward"
+    gbk = gbk.cpu().numpy()
     out = out.float().cpu().numpy()
     lse = lse.cpu().numpy()
     pos = sample_positions(w.n)
-    bsel = [0] if big else list(range(w.batch))
+    bsel = [0] if w.batch * w.n > 65536 else list(range(w.batch))
     for h in heads:
         xs, vs = x[bsel][:, h:h + 1], v[bsel][:, h:h + 1]
-        ro, rl = oracle.forward_sampled(xs, vs, bk[bsel][:, h:h + 1], w.n_buckets, w.chunk,
-                                        w.causal, pos)
+        ref_bk, _ = oracle.hash_all(xs, R)
+        np.testing.assert_array_equal(gbk[bsel][:, h:h + 1], ref_bk,
+                                      err_msg=f"{w.name} h{h}: bucket ids")
+        ro, rl = oracle.forward_sampled(xs, vs, ref_bk, w.n_buckets, w.chunk, w.causal, pos)
         check_close(out[bsel][:, h:h + 1][:, :, pos], ro, w.dtype, f"{w.name} h{h} out")
         check_close(lse[bsel][:, h:h + 1][:, :, :, pos], rl, w.dtype, f"{w.name} h{h} lse")
+
+
+def test_forward_tie_moves_histogram_count():
+    """Tie-built inputs on which the tensor-core screen and the definition pick
+    different buckets inside a forward. Column 3 of every rotation is the
+    negation of column 2, so p_3 = -p_2 exactly. For tokens near -R_r[:, 2],
+    p_2 < 0 has the largest magnitude: the screen takes column 2 with its sign
+    (bucket nb/2 + 2) while the first index of [p ; -p] attaining the maximum
+    is 3 (+p_3). The fp64 re-decision changes the bucket and moves the token's
+    count between the sort's tile histograms; the whole output must then equal
+    the oracle's forward, which hashes on its own."""
+    w = I.Workload("tie-forward", 1, 2, 4096, 64, 64, 64, 2, True, "bf16")
+    x, v = I.make_qkv(w)
+    R = I.make_rotations(w)
+    R[:, :, 3] = -R[:, :, 2]
+    g = torch.Generator().manual_seed(17)
+    for h in range(w.heads):
+        r = h % w.rounds  # head h plants its ties in round h % rounds
+        idx = torch.arange(h, w.n, 3)
+        noise = 0.05 * torch.randn(len(idx), w.d, generator=g)
+        x[0, h, idx] = (-R[r, :, 2].float() + noise).to(torch.bfloat16)
+    ref_out, ref_lse, ref_bk = oracle.forward(x, v, R, w.chunk, w.causal)
+    half = w.n_buckets // 2
+    planted = sum(int((ref_bk[0, h, h % w.rounds] == 3).sum()) for h in range(w.heads))
+    assert planted >= w.n // 2, "the planted tokens should hash to bucket 3"
+    xg, vg, Rg = to_gpu(x, v, R)
+    desc = lb.make_desc(1, 2, w.n, w.d, w.n_buckets, w.chunk, w.rounds, True, torch.bfloat16)
+    ws = lb.workspace(desc, xg.device)
+    out, lse = lb.lsh_attn_forward(xg, vg, Rg, n_buckets=w.n_buckets, chunk=w.chunk,
+                                   causal=True, ws=ws)
+    diag = lb.lsh_attn_get_diag(ws)
+    assert diag["status"] == 0
+    assert diag["hash_refined"] >= planted, diag
+    gbk = lb.lsh_attn_hash(xg, Rg, w.n_buckets).cpu().numpy()
+    np.testing.assert_array_equal(gbk, ref_bk)
+    assert not (gbk == half + 2).all()
+    check_close(out.float().cpu().numpy(), ref_out, "bf16", "tie-forward out")
+    check_close(lse.cpu().numpy(), ref_lse, "bf16", "tie-forward lse")
 
 
 # --------------------------------------------------------------------------
@@ -345,6 +396,61 @@ def test_hash_exact_ties_bit_exact(d, nb):
     diag = lb.lsh_attn_get_diag(ws)
     assert diag["status"] == 0
     assert diag["hash_refined"] >= 16  # at least the zero rows went through fp64
+
+
+NEAR_TIE_CASES = [(64, 64), (64, 2048), (128, 256), (128, 1024), (64, 4096)]
+
+
+@pytest.mark.parametrize("d,nb", NEAR_TIE_CASES, ids=[f"d{d}-nb{nb}" for d, nb in NEAR_TIE_CASES])
+def test_hash_near_ties_stress(d, nb):
+    """Top-two margins planted across the band where an error in the
+    tensor-core screen's bound would show: for column pairs (a, b) of R, column
+    b equals column a except at one row k*, where it differs by delta. A token
+    x = s R[:, a] + noise with x[k*] = t has p_b - p_a = t delta exactly, while
+    |p_a| ~ d leads every other column; t is drawn log-uniformly so that the
+    relative margin (margin / max|p|) spans about 1e-10 .. 1e-3. Pairs straddle
+    16-column batch edges, an MMA chunk edge (192 columns) and the last
+    columns. Every bucket id must equal the oracle's bit for bit."""
+    n, rounds = 4096, 2
+    w = I.Workload("near-ties", 1, 2, n, d, nb, 64, rounds, True, "bf16")
+    R = I.make_rotations(w).float()
+    half = nb // 2
+    pairs = [(a, a + 1) for a in (0, 15, 47, 63, 191, 383, half - 2) if a + 1 < half]
+    pairs = sorted(set(pairs))
+    g = torch.Generator().manual_seed(23)
+    kstar = 5
+    for r in range(rounds):
+        for a, b in pairs:
+            R[r, :, b] = R[r, :, a]
+            R[r, kstar, b] = R[r, kstar, a] + 0.25
+    R = R.to(torch.bfloat16)
+    x = torch.empty(1, 2, n, d)
+    for h in range(2):
+        r = h  # head h plants its near ties in round h
+        pick = torch.randint(0, len(pairs), (n,), generator=g)
+        sign = torch.where(torch.rand(n, generator=g) < 0.5, -1.0, 1.0)
+        t = 10.0 ** (-7 + 6 * torch.rand(n, generator=g))
+        t = t * torch.where(torch.rand(n, generator=g) < 0.5, -1.0, 1.0)
+        cols = torch.tensor([a for a, _ in pairs])[pick]
+        xh = sign[:, None] * R[r][:, cols].float().T + 0.02 * torch.randn(n, d, generator=g)
+        xh[:, kstar] = t
+        x[0, h] = xh
+    x = x.to(torch.bfloat16)
+    ref, margin = oracle.hash_all(x, R)
+    xg, Rg = to_gpu(x, R)
+    desc = lb.make_desc(1, 2, n, d, nb, 64, rounds, True, torch.bfloat16)
+    ws = lb.workspace(desc, xg.device)
+    got = lb.lsh_attn_hash(xg, Rg, nb, ws=ws).cpu().numpy()
+    # relative margins of the planted rounds cover the band
+    p = torch.einsum("hnd,hdj->hnj", x[0].double(), torch.stack([R[0], R[1]]).double())
+    rel = np.array([margin[0, h, h] / p[h].abs().max(dim=1).values.numpy() for h in range(2)])
+    for lo in (1e-7, 1e-6, 1e-5, 1e-4):
+        assert ((rel >= lo) & (rel < 10 * lo)).sum() >= 50, f"few margins in [{lo}, {10 * lo})"
+    diag = lb.lsh_attn_get_diag(ws)
+    print(f"d{d} nb{nb}: {diag['hash_refined']} re-decided; relative margins "
+          f"{np.percentile(rel, [1, 50, 99])}")
+    assert diag["status"] == 0
+    np.testing.assert_array_equal(got, ref)
 
 
 def test_hash_refine_count_is_small():

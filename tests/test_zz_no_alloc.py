@@ -43,3 +43,18 @@ def test_noalloc_sort_rejects_problems_beyond_its_scratch():
     assert e.value.status == 2  # LSH_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert (perm == -7).all()
+
+
+def test_noalloc_sort_clamps_out_of_range_ids_silently():
+    """Ids outside [0, nb) are clamped on this path (no status is readable):
+    the permutation is that of the clamped ids."""
+    w = I.BF16_SHORT
+    bk = I.make_buckets(w, seed=13)
+    bk[0, 0, 0, 5] = w.n_buckets + 3
+    bk[1, 7, 1, 100] = -4
+    bk[0, 3, 1, 0] = 1 << 30
+    clamped = bk.clamp(0, w.n_buckets - 1)
+    got = lb.lsh_attn_sort_noalloc(bk.cuda(), w.n_buckets)
+    ref = lb.lsh_attn_sort(clamped.cuda(), w.n_buckets, d=w.d, dtype=I.torch_dtype(w.dtype))
+    torch.cuda.synchronize()
+    assert torch.equal(got, ref)
