@@ -19,7 +19,7 @@ LSH_F32, LSH_BF16 = 0, 1
 PROFILE_EVENTS = 10  # LSH_ATTN_PROFILE_EVENTS
 #: what ends at each profiling event after the first
 PROFILE_KERNELS = ("hash_prep", "hash_mma", "hash_refine", "sort_hist", "sort_scan",
-                   "sort_rank", "row_gather", "chunk_attention", "unsort_merge")
+                   "sort_rank", "gather_or_norm", "chunk_attention", "unsort_merge")
 _DTYPES = {torch.float32: LSH_F32, torch.bfloat16: LSH_BF16}
 
 #: every symbol the header declares

@@ -1,5 +1,7 @@
 // Chunked shared-QK attention on the 5th-generation tensor cores (bf16 in,
-// fp32 accumulate), chunk m = 64, as a warp-specialised pipeline.
+// fp32 accumulate), chunk m = 64, reading the rows of x and v by the sort's
+// permutation straight from position order: no sorted copies of x and v are
+// ever written.
 //
 // "Reformer summary" (ttnews.xyz), §局部敏感哈希注意力 (chunks of m in the
 // sorted order), §共享QK中的自掩碼 (self-mask); "Reformer: LSH attention and
@@ -9,27 +11,41 @@
 // Work unit: a pair of chunks (c0, c0+1) of one (batch, head, round). Its 128
 // queries are slots [64 c0, 64 c0 + 128) and its key window is slots
 // [64 (c0-1), 64 (c0+2)): the queries are rows 64..191 of the key tile.
+// Units are numbered (batch, head) first, then chunk pair, then round, and
+// CTA c of G takes units c, c + G, c + 2G, ...: at any time the CTAs work on
+// neighbouring units of one (batch, head), so every round reads that head's
+// rows while they sit in L2 and HBM delivers each row about once.
 //
-// One persistent CTA per SM walks a contiguous range of units:
-//   warp 0      TMA: x tile, key norms and positions (stage s = unit & 1),
-//               then the v tile; each as soon as its stage is released
-//   warp 1      tcgen05.mma: S(u+1) = Q K^T into TMEM S[s], then O(u) = P V
+// One persistent CTA per SM, 13 warps:
+//   warps 0-1   x loaders: the window's positions (perm) and key norms
+//               (1/||x|| by position) of the next unit are loaded into
+//               registers while the current unit's rows are in flight, then
+//               written to a 4-deep ring of (logit scale, position) per key;
+//               every 16-byte piece of the 192 x rows goes by cp.async to its
+//               place in the 128-byte-swizzled K-major tile (a slot outside
+//               [0, n) reads as zero). When a thread's copies have landed it
+//               fences them for the async proxy (the tensor cores read shared
+//               memory through it) and arrives.
+//   warps 2-3   v loaders: the same for the v rows, at the positions of the
+//               ring, into the tile of the P.V product.
+//   warp 4      tcgen05.mma: S(u+1) = Q K^T into TMEM S[s], then O(u) = P V
 //               with P read from TMEM, so S of the next unit is ready when
-//               the softmax warps finish the current one
-//   warps 2..5  softmax, one query row per thread, one pass: logits in log2
+//               the softmax warps finish the current one. The x tile is free
+//               again as soon as S is computed (the ring keeps the metadata).
+//   warps 5-8   softmax, one query row per thread, one pass: logits in log2
 //               units are bounded by ||q|| log2(e) / sqrt(d) (keys have unit
 //               length), which serves as the stabiliser, so every probability
 //               is exp2(l - bound) <= 1 and is written to TMEM (bf16, over the
 //               dead S columns) as soon as it is computed; the row sum goes to
 //               the epilogue. A row whose only visible key is itself (the -1e5
 //               self logit) is flagged: its output is v of the query itself.
-//   warps 6..9  epilogue: O from TMEM, divided by the row sum, rounded to
-//               bf16, staged per warp in a 4 KB swizzled buffer (32 rows x 64
-//               columns) and written by TMA bulk stores (slot order), so every
-//               128-byte line leaves the SM whole; the softmax writes lse at
-//               the query's position. Each round's output is kept in bf16: its
-//               rounding (relative 2^-9, before a convex combination over the
-//               rounds) is of the size of the final bf16 rounding of out.
+//   warps 9-12  epilogue: O from TMEM, divided by the row sum and packed to
+//               bf16 (the accumulator is released before the stores), staged
+//               per warp in a 4 KB swizzled buffer (32 rows x 64 columns) and
+//               written by TMA bulk stores (slot order); the softmax writes lse
+//               at the query's position. Each round's output is kept in bf16:
+//               its rounding (relative 2^-9, before a convex combination over
+//               the rounds) is of the size of the final bf16 rounding of out.
 // TMEM: S[0] = [0, 192), S[1] = [192, 384), O = [384, 384 + d).
 #pragma once
 
@@ -40,22 +56,22 @@ namespace lsh {
 
 constexpr int kAttnM = 64;      // chunk length served by this kernel
 constexpr int kAttnKeys = 192;  // key window of a pair of chunks
-constexpr int kAttnWarps = 10;
+constexpr int kAttnWarps = 13;
 constexpr int kAttnStats = 4;   // row-sum slots between softmax and epilogue
+constexpr int kAttnRing = 4;    // metadata ring depth
 // Above this bound (log2 units) the stabiliser could push exp2 below the
 // normal range: those rows use their exact maximum instead.
 constexpr float kAttnBoundMax = 60.f;
 
 struct AttnTcArgs {
-  const float* invnorm;        // [S][n] 1/||x|| of the sorted rows (0 for a zero row)
+  const __nv_bfloat16* x;      // [BH][n][d] position order
+  const __nv_bfloat16* v;      // [BH][n][d] position order
+  const float* pinv;           // [BH][n] 1/||x|| by position (0 for a zero row)
   const int32_t* perm;         // [S][n] position of each slot
-  const __nv_bfloat16* vs;     // [S][n][d] sorted v rows (self-only rows copy theirs)
-  __nv_bfloat16* out_r;        // [S][n][d] each round's output in slot order (TMA stores)
   float* lse;                  // [S][n] each round's lse by position (the caller's output)
   WsHeader* hdr;
-  int n, causal, pairs_per_seg;
-  int64_t pairs;               // S * pairs_per_seg
-  int64_t pairs_per_cta;
+  int n, rounds, pairs_per_seg;
+  int64_t units;               // BH * pairs_per_seg * rounds
 };
 
 // 2^x by the hardware's approximate base-2 exponential (relative error near
@@ -74,51 +90,50 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnWarps * 32, 1)
-    k_attn_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmv,
-              const __grid_constant__ CUtensorMap tmo, AttnTcArgs a) {
+    k_attn_tc(const __grid_constant__ CUtensorMap tmo, AttnTcArgs a) {
   using namespace sm100;
   constexpr int KH = D / 64;
   constexpr uint32_t BOX = kAttnKeys * 128;
   constexpr uint32_t TILE = KH * BOX;
+  constexpr int CPR = KH * 8;       // 16-byte pieces per row
+  constexpr int RSTEP = 64 / CPR;   // rows between a loader thread's pieces
   constexpr float kLog2e = 1.4426950408889634f;
   constexpr int kNoKey = 0x7fffffff;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* xt = base;                                          // [2][KH][192][128 B]
-  unsigned char* vt = base + 2 * TILE;                               // [2][KH][192][128 B]
-  unsigned char* ostage = base + 4 * TILE;                           // [4 warps][32][128 B]
-  float* kinv = reinterpret_cast<float*>(ostage + 4 * 32 * 128);     // [2][192]
-  int32_t* kpos = reinterpret_cast<int32_t*>(kinv + 2 * kAttnKeys);  // [2][192]
-  float2* ktab = reinterpret_cast<float2*>(kpos + 2 * kAttnKeys);    // [2][192] (scale, pos)
-  float* rstat = reinterpret_cast<float*>(ktab + 2 * kAttnKeys);     // [4][128] 1/sum
+  unsigned char* xt = base;                                           // [2][KH][192][128 B]
+  unsigned char* vt = base + 2 * TILE;                                // [2][KH][192][128 B]
+  unsigned char* ostage = base + 4 * TILE;                            // [4 warps][32][128 B]
+  float2* ktab = reinterpret_cast<float2*>(ostage + 4 * 32 * 128);    // [ring][192] (scale, pos)
+  float* rstat = reinterpret_cast<float*>(ktab + kAttnRing * kAttnKeys);  // [4][128] 1/sum
   uint64_t* bars = reinterpret_cast<uint64_t*>(rstat + kAttnStats * 128);
-  uint64_t* xfull = bars + 0;    // [2] tx: x tile + metadata
-  uint64_t* xfree = bars + 2;    // [2] S MMA done + 4 softmax warps done with the metadata
-  uint64_t* vfull = bars + 4;    // [2]
-  uint64_t* vfree = bars + 6;    // [2] PV MMA done
+  uint64_t* xfull = bars + 0;    // [2] x rows landed (64 x-loader threads)
+  uint64_t* xfree = bars + 2;    // [2] S MMA done with the x tile
+  uint64_t* vfull = bars + 4;    // [2] v rows landed (64 v-loader threads)
+  uint64_t* vfree = bars + 6;    // [2] PV MMA done with the v tile
   uint64_t* sfull = bars + 8;    // [2] S MMA done
   uint64_t* pready = bars + 10;  // [2] P written (4 softmax warps)
   uint64_t* sfree = bars + 12;   // [2] PV MMA done with P
   uint64_t* ofull = bars + 14;   // PV MMA done
   uint64_t* ofree = bars + 15;   // 4 epilogue warps done reading O
   uint64_t* statf = bars + 16;   // [4] row sums written (4 softmax warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 21);
-  uint64_t* drain = bars + 22;   // MMA issuer: every issued MMA has completed
-  volatile int* drain_fail = reinterpret_cast<volatile int*>(bars + 23);
+  uint64_t* mfull = bars + 20;   // [ring] metadata written (64 x-loader threads)
+  uint64_t* mfree = bars + 24;   // [ring] 4 softmax warps + 2 v-loader warps done with it
+  uint64_t* drain = bars + 28;   // MMA issuer: every issued MMA has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 29);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 30);
+  volatile int* drain_fail = reinterpret_cast<volatile int*>(bars + 31);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t u0 = blockIdx.x * a.pairs_per_cta;
-  const int64_t u1 = min(a.pairs, u0 + a.pairs_per_cta);
-  if (u0 >= u1) return;  // uniform across the CTA
-  const int nu = (int)(u1 - u0);
+  if ((int64_t)blockIdx.x >= a.units) return;  // uniform across the CTA
+  const int nu = (int)((a.units - 1 - blockIdx.x) / gridDim.x) + 1;
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(xfull + i, 1);
-      mbar_init(xfree + i, 1 + 4);
-      mbar_init(vfull + i, 1);
+      mbar_init(xfull + i, 64);
+      mbar_init(xfree + i, 1);
+      mbar_init(vfull + i, 64);
       mbar_init(vfree + i, 1);
       mbar_init(sfull + i, 1);
       mbar_init(pready + i, 4);
@@ -127,63 +142,109 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     mbar_init(ofull, 1);
     mbar_init(ofree, 4);
     for (int i = 0; i < kAttnStats; ++i) mbar_init(statf + i, 4);
+    for (int i = 0; i < kAttnRing; ++i) {
+      mbar_init(mfull + i, 64);
+      mbar_init(mfree + i, 4 + 2);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     *drain_fail = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 4) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_o = tmem + 384;
+  const float c_scale = kLog2e / sqrtf((float)D);
 
   auto fail = [&]() {
     record_status(a.hdr, 5u /* LSH_ERR_TIMEOUT */);
     *abort_flag = 1;
   };
-  auto unit_seg = [&](int i) { return (u0 + i) / a.pairs_per_seg; };
-  auto unit_c0 = [&](int i) { return (int)((u0 + i) % a.pairs_per_seg) * 2; };
+  // (batch-head, segment, first chunk) of this CTA's unit i
+  auto unit_of = [&](int i, int64_t& bh, int64_t& seg, int& c0) {
+    const int64_t u = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+    const int64_t per_bh = (int64_t)a.pairs_per_seg * a.rounds;
+    bh = u / per_bh;
+    const int rem = (int)(u - bh * per_bh);
+    const int pair = rem / a.rounds;
+    seg = bh * a.rounds + (rem - pair * a.rounds);
+    c0 = 2 * pair;
+  };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmx);
-      prefetch_tensormap(&tmv);
-      bool ok = true;
-      int lastx[2] = {-1, -1}, lastv[2] = {-1, -1};  // last phase issued per stage
-      for (int i = 0; ok && i < nu && !*abort_flag; ++i) {
-        const int s = i & 1, k = i >> 1;
-        const int64_t seg = unit_seg(i);
-        const int k0 = (unit_c0(i) - 1) * kAttnM;  // first key slot (may be < 0)
-        const int row = (int)(seg * a.n) + k0;
-        if (k > 0 && !mbar_wait(xfree + s, (k - 1) & 1)) { ok = false; break; }
-        const int lo = max(0, k0), hi = min(a.n, k0 + kAttnKeys);
-        const uint32_t mbytes = (uint32_t)(hi - lo) * 4;
-        mbar_expect_tx(xfull + s, TILE + 2 * mbytes);
-        for (int kh = 0; kh < KH; ++kh)
-          tma_load_2d(xt + s * TILE + kh * BOX, &tmx, xfull + s, kh * 64, row);
-        bulk_copy_g2s(kinv + s * kAttnKeys + (lo - k0), a.invnorm + seg * a.n + lo, mbytes,
-                      xfull + s);
-        bulk_copy_g2s(kpos + s * kAttnKeys + (lo - k0), a.perm + seg * a.n + lo, mbytes,
-                      xfull + s);
-        lastx[s] = k;
-        if (k > 0 && !mbar_wait(vfree + s, (k - 1) & 1)) { ok = false; break; }
-        mbar_expect_tx(vfull + s, TILE);
-        for (int kh = 0; kh < KH; ++kh)
-          tma_load_2d(vt + s * TILE + kh * BOX, &tmv, vfull + s, kh * 64, row);
-        lastv[s] = k;
+  if (warp < 4) {
+    // ------------------------------------------------------------ loaders
+    const bool xl = warp < 2;      // x loaders write the ring; v loaders read it
+    const int lt = tid & 63;       // rank among this loader pair of warps
+    const unsigned char* src0 = reinterpret_cast<const unsigned char*>(xl ? a.x : a.v);
+    unsigned char* tiles = xl ? xt : vt;
+    uint64_t* full = xl ? xfull : vfull;
+    uint64_t* tfree = xl ? xfree : vfree;
+    const int piece = lt % CPR;    // this thread's 16-byte piece of every row it copies
+    const int kh = piece >> 3, cc = piece & 7;
+    // x loaders: positions and logit scales of the next unit's window (rows
+    // lt, lt + 64, lt + 128), loaded a unit ahead
+    int pj[3];
+    float sj[3];
+    auto fetch = [&](int i) {
+      int64_t bh, seg;
+      int c0;
+      unit_of(i, bh, seg, c0);
+      const int k0 = (c0 - 1) * kAttnM;
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {
+        const int ks = k0 + lt + 64 * q;
+        pj[q] = (ks >= 0 && ks < a.n) ? __ldg(a.perm + seg * a.n + ks) : kNoKey;
       }
-      if (!ok) fail();
-      // No copy may still be writing this CTA's shared memory when it exits:
-      // wait (bounded) for the last phase issued on every stage.
-      for (int s = 0; s < 2; ++s)
-        if ((lastx[s] >= 0 && !mbar_wait(xfull + s, lastx[s] & 1)) ||
-            (lastv[s] >= 0 && !mbar_wait(vfull + s, lastv[s] & 1)))
-          *drain_fail = 1;
+#pragma unroll
+      for (int q = 0; q < 3; ++q)
+        sj[q] = pj[q] != kNoKey ? __ldg(a.pinv + bh * a.n + pj[q]) * c_scale : 0.f;
+    };
+    if (xl) fetch(0);
+    for (int i = 0; i < nu; ++i) {
+      const int s = i & 1, k = i >> 1, m = i & (kAttnRing - 1), km = i / kAttnRing;
+      bool got;
+      if (xl)  // ring slot m free (unit i - 4 done with it), x tile s free (S of unit i - 2)
+        got = (km == 0 || mbar_wait(mfree + m, (km - 1) & 1)) &&
+              (k == 0 || mbar_wait(tfree + s, (k - 1) & 1));
+      else     // ring slot m written for unit i, v tile s free (PV of unit i - 2)
+        got = mbar_wait(mfull + m, km & 1) && (k == 0 || mbar_wait(tfree + s, (k - 1) & 1));
+      if (!got) fail();
+      // both warps of the pair stop together (a failure anywhere sets abort_flag)
+      if (bar_sync_any(2 + (xl ? 0 : 1), 64, !got || *abort_flag)) break;
+      float2* kt = ktab + m * kAttnKeys;
+      if (xl) {
+#pragma unroll
+        for (int q = 0; q < 3; ++q) kt[lt + 64 * q] = make_float2(sj[q], __int_as_float(pj[q]));
+        bar_sync_any(2, 64, false);  // the pair's ring entries are written
+        mbar_arrive(mfull + m);
+      }
+      int64_t bh, seg;
+      int c0;
+      unit_of(i, bh, seg, c0);
+      const unsigned char* rows = src0 + (bh * a.n) * (int64_t)(D * 2) + piece * 16;
+      unsigned char* dst = tiles + s * TILE + kh * BOX;
+#pragma unroll 4
+      for (int row = lt / CPR; row < kAttnKeys; row += RSTEP) {
+        const int pos = __float_as_int(kt[row].y);
+        const bool valid = pos != kNoKey;
+        const unsigned char* src = valid ? rows + (int64_t)pos * (D * 2) : src0;
+        cp_async16_zfill(dst + row * 128 + ((cc ^ (row & 7)) << 4), src, valid);
+      }
+      cp_async_commit();
+      if (!xl) {  // done reading the ring slot
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mfree + m);
+      }
+      if (xl && i + 1 < nu) fetch(i + 1);  // in flight while this unit's rows land
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(full + s);
     }
-  } else if (warp == 1) {
+    cp_async_wait_all();  // nothing of this thread's still writes shared memory at exit
+  } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, kAttnKeys);
@@ -230,39 +291,28 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       mma_commit(drain);
       if (!mbar_wait(drain, 0)) *drain_fail = 1;
     }
-  } else if (warp < 6) {
+  } else if (warp < 9) {
     // ------------------------------------------------------------ softmax
     const int q = warp & 3;       // TMEM lane quadrant
-    const int st = tid - 64;      // 0..127 among the softmax threads
     const int row = q * 32 + lane;
     const int wcol = q < 2 ? 0 : kAttnM;  // first in-window key column
     const uint32_t tl = (uint32_t)(q * 32) << 16;
-    const float c_scale = kLog2e / sqrtf((float)D);
     for (int i = 0; i < nu; ++i) {
-      const int s = i & 1, k = i >> 1;
-      const bool got = mbar_wait(sfull + s, k & 1);
+      const int s = i & 1, k = i >> 1, m = i & (kAttnRing - 1), km = i / kAttnRing;
+      const bool got = mbar_wait(sfull + s, k & 1) && mbar_wait(mfull + m, km & 1);
       if (!got) fail();
       tc_fence_after();
-      const int64_t seg = unit_seg(i);
-      const int c0 = unit_c0(i);
-      const int k0 = (c0 - 1) * kAttnM;
-      // per-key table: logit scale (log2 units) and position; keys outside
-      // [0, n) get a position that every query's test rejects
-      float2* kt = ktab + s * kAttnKeys;
-      for (int j = st; got && j < kAttnKeys; j += 128) {
-        const int ks = k0 + j;
-        const bool valid = ks >= 0 && ks < a.n;
-        kt[j] = make_float2(valid ? kinv[s * kAttnKeys + j] * c_scale : 0.f,
-                            __int_as_float(valid ? kpos[s * kAttnKeys + j] : kNoKey));
-      }
-      const float qinv = kinv[s * kAttnKeys + kAttnM + row];
       // the four softmax warps; a failure seen by any of them stops all four
       // here, so none is left waiting at this barrier
       if (bar_sync_any(1, 128, !got || *abort_flag)) break;
-      if (lane == 0) mbar_arrive(xfree + s);  // metadata of this stage consumed
-      const int qpos = __float_as_int(kt[kAttnM + row].y);
+      int64_t bh, seg;
+      int c0;
+      unit_of(i, bh, seg, c0);
+      const float2* kt = ktab + m * kAttnKeys;
+      const float2 me = kt[kAttnM + row];
+      const int qpos = __float_as_int(me.y);
       // stabiliser: ||q|| log2(e) / sqrt(d) bounds every logit of the row
-      float bound = qinv > 0.f ? c_scale / qinv : 0.f;
+      float bound = me.x > 0.f ? c_scale * c_scale / me.x : 0.f;
       const uint32_t ts = tmem + tl + s * 192;
       auto visible = [&](int pj) {
         if (CAUSAL) return pj < qpos;            // earlier positions only (not self)
@@ -286,8 +336,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       }
       float sum0 = 0.f, sum1 = 0.f;
       // 32-key batches per TMEM wait: two at d = 64, where the softmax paces
-      // the pipeline (more exponents in flight), one at d = 128, where the
-      // registers are spoken for
+      // the pipeline (more exponents in flight), one at d = 128
       constexpr int BPW = D == 64 ? 2 : 1;
 #pragma unroll 1
       for (int b2 = 0; b2 < 4; b2 += BPW) {
@@ -338,6 +387,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       if (lane == 0) {
         mbar_arrive(pready + s);
         mbar_arrive(statf + (i % kAttnStats));
+        mbar_arrive(mfree + m);
       }
     }
   } else {
@@ -351,19 +401,35 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         break;
       }
       tc_fence_after();
-      uint32_t o[D / 32][32];
+      const float inv = rstat[(i % kAttnStats) * 128 + row];
+      // O / sum, packed to bf16 pairs as it leaves TMEM: pk[j] = columns 2j, 2j+1
+      uint32_t pk[D / 2];
 #pragma unroll
-      for (int b = 0; b < D / 32; ++b) tmem_ld32(tm_o + tl + b * 32, o[b]);
-      tmem_wait_ld();
+      for (int b = 0; b < D / 64; ++b) {
+        uint32_t o[2][32];
+        tmem_ld32(tm_o + tl + b * 64, o[0]);
+        tmem_ld32(tm_o + tl + b * 64 + 32, o[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int c = 0; c < 32; c += 2)
+            pk[b * 32 + h * 16 + c / 2] =
+                pack_bf16x2(__uint_as_float(o[h][c]) * inv, __uint_as_float(o[h][c + 1]) * inv);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ofree);
-      const int64_t seg = unit_seg(i);
-      const int qs0 = unit_c0(i) * kAttnM + q * 32;  // first query slot of this warp
+      int64_t bh, seg;
+      int c0;
+      unit_of(i, bh, seg, c0);
+      const int qs0 = c0 * kAttnM + q * 32;  // first query slot of this warp
       if (qs0 < a.n) {  // n % 64 == 0: a warp's 32 rows are all valid or all not
-        const float inv = rstat[(i % kAttnStats) * 128 + row];
-        const uint4* vr = reinterpret_cast<const uint4*>(a.vs + (seg * a.n + qs0 + lane) * (int64_t)D);
-        unsigned char* stg = ostage + (warp - 6) * 32 * 128;
+        const uint4* vr = nullptr;
+        if (inv <= 0.f)  // only the token itself is visible: its own value row
+          vr = reinterpret_cast<const uint4*>(
+              a.v + (bh * a.n + a.perm[seg * a.n + qs0 + lane]) * (int64_t)D);
+        unsigned char* stg = ostage + (warp - 9) * 32 * 128;
 #pragma unroll
         for (int b = 0; b < D / 64; ++b) {  // 64 columns (128 bytes of bf16) per store
           if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
@@ -371,20 +437,12 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
           // row `lane`, 16-byte chunk c (columns 64 b + 8 c ...) goes to slot
           // c ^ (lane % 8) (128-byte swizzle)
           unsigned char* line = stg + lane * 128;
-          if (inv > 0.f) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const uint32_t* src = &o[2 * b + (c >> 2)][8 * (c & 3)];
-              *reinterpret_cast<uint4*>(line + ((c ^ (lane & 7)) << 4)) = make_uint4(
-                  pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv),
-                  pack_bf16x2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv),
-                  pack_bf16x2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv),
-                  pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv));
-            }
-          } else {  // only the token itself is visible: its own value row
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4*>(line + ((c ^ (lane & 7)) << 4)) = vr[b * 8 + c];
+          for (int c = 0; c < 8; ++c) {
+            const uint4 val = vr ? vr[b * 8 + c]
+                                 : make_uint4(pk[b * 32 + 4 * c], pk[b * 32 + 4 * c + 1],
+                                              pk[b * 32 + 4 * c + 2], pk[b * 32 + 4 * c + 3]);
+            *reinterpret_cast<uint4*>(line + ((c ^ (lane & 7)) << 4)) = val;
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -401,7 +459,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   __syncthreads();
   // after a drain that gave up, TMEM is left allocated rather than freed
   // under a running MMA; the status word already records the timeout
-  if (warp == 1 && !*drain_fail) {
+  if (warp == 4 && !*drain_fail) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -409,8 +467,36 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
 
 inline size_t attn_tc_smem(int D) {
   const size_t tile = (size_t)(D / 64) * kAttnKeys * 128;
-  return 1024 + 4 * tile + 4 * 32 * 128 + 2 * kAttnKeys * (4 + 4 + 8) + kAttnStats * 128 * 4 +
-         256;
+  return 1024 + 4 * tile + 4 * 32 * 128 + (size_t)kAttnRing * kAttnKeys * 8 +
+         kAttnStats * 128 * 4 + 256;
+}
+
+// 1/||x|| of every row of x [rows][D] (bf16), for the attention's key scales
+// when the hash did not produce them: a group of D / 8 lanes per row, one
+// 16-byte piece per lane, the square sum reduced inside the group.
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_row_invnorm(const __nv_bfloat16* __restrict__ x, float* __restrict__ pinv, int64_t rows) {
+  constexpr int L = D / 8;  // lanes per row: 8 or 16
+  const int gl = threadIdx.x % L;
+  const int64_t stride = (int64_t)gridDim.x * (blockDim.x / L);
+  // the same trip count for every lane of a warp (the group shuffles below)
+  const int64_t first = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / L;
+  const int64_t warp_first = first - (threadIdx.x & 31) / L;
+  for (int64_t r0 = warp_first; r0 < rows; r0 += stride) {
+    const int64_t r = r0 + (threadIdx.x & 31) / L;
+    float ss = 0.f;
+    if (r < rows) {
+      const uint4 u = *reinterpret_cast<const uint4*>(x + r * D + gl * 8);
+      float f[8];
+      Vec16<__nv_bfloat16>::unpack(u, f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+    }
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (r < rows && gl == 0) pinv[r] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+  }
 }
 
 }  // namespace lsh

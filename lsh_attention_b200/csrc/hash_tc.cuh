@@ -242,6 +242,7 @@ struct HashTcArgs {
   int64_t cap;        // BH * n
   WsHeader* hdr;      // rnorm bits in hdr->pad[0, 16), queue lengths in hdr->pad[16, 32)
   int32_t* hist;      // the sort's [seg][nb][sort_tiles] counts (zeroed), or null
+  float* pinv;        // [BH][n] 1/||x|| by position (the attention's key scales), or null
   int n, nb, rounds, tiles_per_seq, tiles, ctas_per_group;
   int sort_tile, sort_tiles;  // tokens per sort tile, sort tiles per sequence
 };
@@ -577,6 +578,8 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
             float sst = 0.f;
 #pragma unroll
             for (int o_ = 0; o_ < PO; ++o_) sst += sslot[o_ * 32];
+            if (a.pinv != nullptr && r == 0)  // once per token, from the first round
+              a.pinv[(int64_t)bh * a.n + t] = sst > 0.f ? 1.0f / sqrtf(sst) : 0.f;
             const float xnorm = sqrtf(sst) * 1.0001f;
             const float tau = kTieFactor * (float)D * 1.1920929e-7f * xnorm * rn_s[r];
             const int bucket = idx + (sv < 0.f ? p.half : 0);

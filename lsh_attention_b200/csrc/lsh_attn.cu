@@ -23,7 +23,8 @@ namespace {
 using namespace lsh;
 
 struct Layout {
-  size_t header, buckets, perm, inv, invnorm, lse_s, hist, xs, vs, out_s, rt, refine, total;
+  size_t header, buckets, perm, inv, invnorm, pinv, lse_s, hist, xs, vs, out_s, rt, refine,
+      total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -33,7 +34,14 @@ struct Dims {
   int64_t BH, S;  // (batch, head) pairs; segments = BH * rounds
   int esize;
   int tiles;
+  bool attention;  // the call runs the chunked attention (the forward)
 };
+
+// bf16, chunk 64: the tcgen05 kernel, which reads x and v rows by perm.
+inline bool attn_tc_supported(const Dims& D) {
+  return D.dtype == LSH_BF16 && D.m == kAttnM && D.n % kAttnM == 0 &&
+         D.S * (int64_t)D.n < (int64_t(1) << 31);
+}
 
 // `attention`: the call runs the chunked attention, so the chunk length must
 // be in the supported set; hash and sort ignore it beyond chunk >= 1.
@@ -61,6 +69,7 @@ lsh_status check_desc(const lsh_attn_desc* desc, Dims* D, bool attention) {
   D->BH = (int64_t)q.batch * q.heads;
   D->S = D->BH * q.rounds;
   D->esize = q.dtype == LSH_BF16 ? 2 : 4;
+  D->attention = attention;
   const int tile = sort_tile(q.n_buckets);
   D->tiles = (q.n + tile - 1) / tile;
   if (D->S * (int64_t)q.n * q.d >= (int64_t(1) << 40)) return LSH_ERR_UNSUPPORTED;
@@ -77,16 +86,22 @@ Layout layout_of(const Dims& D) {
     return at;
   };
   const size_t sn = (size_t)D.S * D.n;
+  // the forward's attention reads x and v by perm on the tensor-core path
+  // (key scales by position: pinv) and sorted copies otherwise (xs, vs, and
+  // key scales by slot: invnorm); hash and sort calls need neither
+  const bool tc = D.attention && attn_tc_supported(D);
+  const bool copies = D.attention && !tc;
   L.header = take(sizeof(WsHeader));
   L.buckets = take(sn * 4);
   L.perm = take(sn * 4);
   L.inv = take(sn * 4);
-  L.invnorm = take(sn * 4);
+  L.invnorm = take(tc ? 0 : sn * 4);  // also written by lsh_attn_sort's row gather
+  L.pinv = take(tc ? (size_t)D.BH * D.n * 4 : 0);
   L.lse_s = take(sn * 4);
   L.hist = take((size_t)D.S * D.nb * D.tiles * 4);
-  L.xs = take(sn * D.d * D.esize);
-  L.vs = take(sn * D.d * D.esize);
-  L.out_s = take(sn * D.d * D.esize);  // each round's output rows, in the input type
+  L.xs = take(copies ? sn * D.d * D.esize : 0);
+  L.vs = take(copies ? sn * D.d * D.esize : 0);
+  L.out_s = take(D.attention ? sn * D.d * D.esize : 0);  // each round's output, input type
   const HashTcPlan hp = hash_tc_plan(D.d, D.nb, D.rounds);
   L.rt = take((size_t)D.rounds * hp.ch * hp.nc * D.d * 2);  // R transposed (bf16 hash)
   L.refine = take(sn * 8);                             // near-tie queue of the bf16 hash
@@ -166,13 +181,16 @@ lsh_status launch_hash_exact(const Dims& D, const void* x, const void* R, int32_
 
 // bf16: tcgen05 projection + top-2 screen, fp64 re-decision of near ties.
 // hist: when not null, the sort's tile histograms are counted by the hash
-// (and *hist_done set); otherwise the sort counts them itself.
+// (and *hist_done set); otherwise the sort counts them itself. pinv: when not
+// null, 1/||x|| by position is written too (and *pinv_done set).
 lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const void* R,
                           int32_t* buckets, void* ws, cudaStream_t st, void* const* ev,
-                          int32_t* hist = nullptr, bool* hist_done = nullptr) {
+                          int32_t* hist = nullptr, bool* hist_done = nullptr,
+                          float* pinv = nullptr, bool* pinv_done = nullptr) {
   const HashTcPlan p = hash_tc_plan(D.d, D.nb, D.rounds);
   lsh_status s;
   if (hist_done) *hist_done = false;
+  if (pinv_done) *pinv_done = false;
   if (p.group == 0) {
     if ((s = mark(ev, 1, st)) != LSH_OK) return s;
     if ((s = launch_hash_exact(D, x, R, buckets, st, true)) != LSH_OK) return s;
@@ -203,6 +221,7 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
   a.tiles_per_seq = (D.n + kHashTile - 1) / kHashTile;
   a.tiles = (int)(D.BH * a.tiles_per_seq);
   a.hist = hist;
+  a.pinv = pinv;
   a.sort_tile = sort_tile(D.nb);
   a.sort_tiles = D.tiles;
   if (hist != nullptr &&
@@ -241,14 +260,18 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
                                            hdr, hist, a.sort_tile, a.sort_tiles);
   if ((s = last_cuda()) != LSH_OK) return s;
   if (hist_done) *hist_done = hist != nullptr;
+  if (pinv_done) *pinv_done = pinv != nullptr;
   return mark(ev, 3, st);
 }
 
 lsh_status launch_hash(const Dims& D, const Layout& L, const void* x, const void* R,
                        int32_t* buckets, void* ws, cudaStream_t st, void* const* ev = nullptr,
-                       int32_t* hist = nullptr, bool* hist_done = nullptr) {
-  if (D.dtype == LSH_BF16) return launch_hash_tc(D, L, x, R, buckets, ws, st, ev, hist, hist_done);
+                       int32_t* hist = nullptr, bool* hist_done = nullptr,
+                       float* pinv = nullptr, bool* pinv_done = nullptr) {
+  if (D.dtype == LSH_BF16)
+    return launch_hash_tc(D, L, x, R, buckets, ws, st, ev, hist, hist_done, pinv, pinv_done);
   if (hist_done) *hist_done = false;
+  if (pinv_done) *pinv_done = false;
   lsh_status s;
   if ((s = mark(ev, 1, st)) != LSH_OK) return s;
   if ((s = launch_hash_exact(D, x, R, buckets, st, false)) != LSH_OK) return s;
@@ -289,8 +312,7 @@ lsh_status launch_sort(const Dims& D, const int32_t* buckets, const void* x, con
         perm, static_cast<const T*>(x), static_cast<const T*>(v), static_cast<T*>(xs),
         static_cast<T*>(vs), invnorm, D.n, D.rounds);
   }
-  if ((s = last_cuda()) != LSH_OK) return s;
-  return mark(ev, 7, st);
+  return last_cuda();
 }
 
 template <typename T, int DD, int QPW>
@@ -316,53 +338,55 @@ lsh_status launch_attn_simt(const Dims& D, const void* xs, const void* vs, const
   return launch_attn_simt_q<T, DD, 16>(D, xs, vs, perm, invnorm, out_s, lse_s, st);
 }
 
-// bf16, chunk 64: tcgen05 kernel on pairs of chunks.
-inline bool attn_tc_supported(const Dims& D) {
-  return D.dtype == LSH_BF16 && D.m == kAttnM && D.n % kAttnM == 0 &&
-         D.S * (int64_t)D.n < (int64_t(1) << 31);
-}
-
 template <int DD, bool CAUSAL>
-lsh_status launch_attn_tc_k(const CUtensorMap& tmx, const CUtensorMap& tmv,
-                            const CUtensorMap& tmo, const AttnTcArgs& a, unsigned grid,
+lsh_status launch_attn_tc_k(const CUtensorMap& tmo, const AttnTcArgs& a, unsigned grid,
                             size_t smem, cudaStream_t st) {
   auto kern = k_attn_tc<DD, CAUSAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return LSH_ERR_CUDA;
-  kern<<<grid, kAttnWarps * 32, smem, st>>>(tmx, tmv, tmo, a);
+  kern<<<grid, kAttnWarps * 32, smem, st>>>(tmo, a);
   return last_cuda();
 }
 
-lsh_status launch_attn_tc(const Dims& D, const void* xs, const void* vs, const int32_t* perm,
-                          const float* invnorm, void* out_r, float* lse, WsHeader* hdr,
+// Chunk attention on the tensor cores, rows of x and v read by perm.
+lsh_status launch_attn_tc(const Dims& D, const void* x, const void* v, const int32_t* perm,
+                          const float* pinv, void* out_r, float* lse, WsHeader* hdr,
                           cudaStream_t st) {
-  CUtensorMap tmx, tmv, tmo;
+  CUtensorMap tmo;
   const uint64_t rows = (uint64_t)D.S * D.n;
-  if (!make_tmap_bf16_2d(&tmx, xs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys) ||
-      !make_tmap_bf16_2d(&tmv, vs, D.d, rows, (uint64_t)D.d * 2, 64, kAttnKeys) ||
-      !make_tmap_bf16_2d(&tmo, out_r, D.d, rows, (uint64_t)D.d * 2, 64, 32))
-    return LSH_ERR_CUDA;
+  if (!make_tmap_bf16_2d(&tmo, out_r, D.d, rows, (uint64_t)D.d * 2, 64, 32)) return LSH_ERR_CUDA;
   AttnTcArgs a;
-  a.invnorm = invnorm;
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.pinv = pinv;
   a.perm = perm;
-  a.vs = static_cast<const __nv_bfloat16*>(vs);
-  a.out_r = static_cast<__nv_bfloat16*>(out_r);
   a.lse = lse;
   a.hdr = hdr;
   a.n = D.n;
-  a.causal = D.causal;
+  a.rounds = D.rounds;
   a.pairs_per_seg = (D.n / kAttnM + 1) / 2;
-  a.pairs = D.S * a.pairs_per_seg;
-  const int64_t ctas_max = (int64_t)sm_count();
-  a.pairs_per_cta = (a.pairs + ctas_max - 1) / ctas_max;
-  const unsigned grid = (unsigned)((a.pairs + a.pairs_per_cta - 1) / a.pairs_per_cta);
+  a.units = D.S * a.pairs_per_seg;
+  const unsigned grid = (unsigned)std::min<int64_t>(a.units, sm_count());
   const size_t smem = attn_tc_smem(D.d);
   if (D.d == 64)
-    return D.causal ? launch_attn_tc_k<64, true>(tmx, tmv, tmo, a, grid, smem, st)
-                    : launch_attn_tc_k<64, false>(tmx, tmv, tmo, a, grid, smem, st);
-  return D.causal ? launch_attn_tc_k<128, true>(tmx, tmv, tmo, a, grid, smem, st)
-                  : launch_attn_tc_k<128, false>(tmx, tmv, tmo, a, grid, smem, st);
+    return D.causal ? launch_attn_tc_k<64, true>(tmo, a, grid, smem, st)
+                    : launch_attn_tc_k<64, false>(tmo, a, grid, smem, st);
+  return D.causal ? launch_attn_tc_k<128, true>(tmo, a, grid, smem, st)
+                  : launch_attn_tc_k<128, false>(tmo, a, grid, smem, st);
+}
+
+// 1/||x|| by position, when the hash has not written it.
+lsh_status launch_row_invnorm(const Dims& D, const void* x, float* pinv, cudaStream_t st) {
+  const int64_t rows = D.BH * D.n;
+  const int per_block = 256 / (D.d / 8);
+  const unsigned blocks =
+      (unsigned)std::min<int64_t>((rows + per_block - 1) / per_block, (int64_t)8 * sm_count());
+  if (D.d == 64)
+    k_row_invnorm<64><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), pinv, rows);
+  else
+    k_row_invnorm<128><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), pinv, rows);
+  return last_cuda();
 }
 
 template <typename T, int DD>
@@ -382,13 +406,15 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
                          const void* R, const int32_t* buckets, void* out, float* lse, void* ws,
                          cudaStream_t st, void* const* ev) {
   WsHeader* hdr = at<WsHeader>(ws, L.header);
+  const bool tc = attn_tc_supported(D);
+  float* pinv = tc ? at<float>(ws, L.pinv) : nullptr;
   lsh_status s;
   if ((s = mark(ev, 0, st)) != LSH_OK) return s;
-  bool hist_ready = false;
+  bool hist_ready = false, pinv_ready = false;
   if (!buckets) {
     int32_t* bk = at<int32_t>(ws, L.buckets);
-    if ((s = launch_hash(D, L, x, R, bk, ws, st, ev, at<int32_t>(ws, L.hist), &hist_ready)) !=
-        LSH_OK)
+    if ((s = launch_hash(D, L, x, R, bk, ws, st, ev, at<int32_t>(ws, L.hist), &hist_ready, pinv,
+                         &pinv_ready)) != LSH_OK)
       return s;
     buckets = bk;
   } else {
@@ -397,18 +423,27 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
   }
   int32_t* perm = at<int32_t>(ws, L.perm);
   int32_t* inv = at<int32_t>(ws, L.inv);
-  float* invnorm = at<float>(ws, L.invnorm);
-  void* xs = at<unsigned char>(ws, L.xs);
-  void* vs = at<unsigned char>(ws, L.vs);
   T* out_r = at<T>(ws, L.out_s);  // each round's output rows, slot order
-  if ((s = launch_sort<T>(D, buckets, x, v, perm, inv, xs, vs, invnorm, at<int32_t>(ws, L.hist),
-                          hdr, st, ev, hist_ready)) != LSH_OK)
-    return s;
-  if (attn_tc_supported(D))
-    s = launch_attn_tc(D, xs, vs, perm, invnorm, out_r, lse, hdr, st);
-  else
+  if (tc) {
+    // ranks only; the attention reads the rows by perm (and the key scales
+    // by position: from the hash, or from the norm pass here)
+    if ((s = launch_sort<T>(D, buckets, x, v, perm, inv, nullptr, nullptr, nullptr,
+                            at<int32_t>(ws, L.hist), hdr, st, ev, hist_ready)) != LSH_OK)
+      return s;
+    if (!pinv_ready && (s = launch_row_invnorm(D, x, pinv, st)) != LSH_OK) return s;
+    if ((s = mark(ev, 7, st)) != LSH_OK) return s;
+    s = launch_attn_tc(D, x, v, perm, pinv, out_r, lse, hdr, st);
+  } else {
+    float* invnorm = at<float>(ws, L.invnorm);
+    void* xs = at<unsigned char>(ws, L.xs);
+    void* vs = at<unsigned char>(ws, L.vs);
+    if ((s = launch_sort<T>(D, buckets, x, v, perm, inv, xs, vs, invnorm,
+                            at<int32_t>(ws, L.hist), hdr, st, ev, hist_ready)) != LSH_OK)
+      return s;
+    if ((s = mark(ev, 7, st)) != LSH_OK) return s;
     s = D.d == 64 ? launch_attn_simt<T, 64>(D, xs, vs, perm, invnorm, out_r, lse, st)
                   : launch_attn_simt<T, 128>(D, xs, vs, perm, invnorm, out_r, lse, st);
+  }
   if (s != LSH_OK) return s;
   if ((s = mark(ev, 8, st)) != LSH_OK) return s;
   s = D.d == 64 ? launch_merge<T, 64>(D, inv, lse, out_r, out, st)

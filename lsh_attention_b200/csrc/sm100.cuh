@@ -193,6 +193,23 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[4][16]) {
       :
       : "memory");
 }
+// 16-byte copy global -> shared through L2 (cp.async: a generic-proxy write,
+// so a reader through the async proxy needs fence_proxy_async_smem after it
+// has landed). When `valid` is false nothing is read and the 16 bytes are
+// zero-filled. Both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until every cp.async this thread issued has landed.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Untiled bulk copy global -> shared (16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes,
                                               uint64_t* bar) {
