@@ -430,6 +430,45 @@ def e2e_overlapped(m: dict, dev, K2: int, world: int) -> tuple[float, int, int]:
     return ms, h2d, d2h
 
 
+DENSE_16K = I.Workload("dense-16k", 1, 8, 16384, 64, 2, 16384, 1, True, "bf16")
+
+
+def dense_comparison(dev, K: int = 20, W: int = 3) -> dict:
+    """Dense shared-QK causal attention against the LSH forward at n = 16K
+    (8 heads, d = 64; LSH with n/64 buckets, chunk 64, 1 to 8 rounds), each
+    timed with CUDA events over K passes after W, on the same seeded inputs."""
+    w = DENSE_16K
+    stream = torch.cuda.current_stream(dev)
+    x_h, v_h = I.make_qkv(w)
+    x, v = x_h.to(dev), v_h.to(dev)
+    out = torch.empty_like(x)
+    lse = torch.empty((w.batch, w.heads, w.n), dtype=torch.float32, device=dev)
+    for _ in range(W):
+        lb.lsh_attn_dense_forward(x, v, causal=True, out=out, lse=lse)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s0.record(stream)
+    for _ in range(K):
+        lb.lsh_attn_dense_forward(x, v, causal=True, out=out, lse=lse)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = s0.elapsed_time(s1) / K
+    # visible (query, key) pairs under the causal mask, QK^T and PV
+    flops = 2 * 2 * (w.n * (w.n + 1) // 2) * w.d * w.heads * w.batch
+    pk, _ = peaks()
+    res = {"config": config_of(w), "dense_ms": round(dense_ms, 4),
+           "dense_TFLOP/s": round(flops / dense_ms / 1e9, 1),
+           "dense_tensor_frac": round(flops / dense_ms / 1e9 / pk["bf16_tflops"], 4),
+           "lsh_ms": {}, "dense_over_lsh": {}}
+    for rounds in (1, 2, 4, 8):
+        wl = I.Workload(f"lsh-16k-r{rounds}", 1, 8, 16384, 64, 256, 64, rounds, True, "bf16")
+        m = measure(wl, dev, K, W)
+        ms = m["total_ms"] / m["K"]
+        res["lsh_ms"][rounds] = round(ms, 4)
+        res["dense_over_lsh"][rounds] = round(dense_ms / ms, 2)
+    return res
+
+
 def run_ours(args, w):
     world, rank, local = dist_setup("nccl")
     torch.cuda.set_device(local)
@@ -454,6 +493,7 @@ def run_ours(args, w):
                            "roofline": rf, "stages": st,
                            "kernels_ms": {kn: round(t, 4) for kn, t in mx["kernel_ms"].items()}}
             del mx
+        extra["dense_baseline"] = dense_comparison(dev)
     if rank != 0:
         return
     stages, roof = roofline_block(w, m["kernel_ms"], total_ms / 1e3)

@@ -191,6 +191,48 @@ lsh_status lsh_attn_selftest_wait_timeout(void *workspace, size_t workspace_byte
 lsh_status lsh_attn_sort_noalloc(const lsh_attn_desc *desc, const int32_t *buckets,
                                  int32_t *perm, void *stream);
 
+/* Workspace bytes lsh_attn_dense_forward needs for `desc` (only batch,
+ * heads, n, d, causal and dtype are read). Writes *bytes. */
+lsh_status lsh_attn_dense_workspace_size(const lsh_attn_desc *desc, size_t *bytes);
+
+/* Dense shared-QK attention, the full-attention baseline the pages compare
+ * LSH attention with ("Reformer: LSH attention and reversible layers",
+ * §三.3): every query attends to every key (causal: every key at an earlier
+ * position) under the same rules as lsh_attn_forward's chunks -- keys scaled
+ * to unit length, logits scaled by 1/sqrt(d), the -1e5 self logit -- so it
+ * equals lsh_attn_forward with one round and one chunk spanning the sequence.
+ *   x, v, out [B][H][n][d] bf16 (LSH_BF16 only, else LSH_ERR_UNSUPPORTED);
+ *   lse [B][H][n] fp32, natural log. Any n >= 1; d in {64, 128};
+ *   B * H * roundup(n, 128) < 2^31. n_buckets, chunk and rounds are ignored.
+ *   workspace: lsh_attn_dense_workspace_size bytes, 256-byte aligned.
+ * Conventions (ownership, asynchrony, errors) as for lsh_attn_forward. */
+lsh_status lsh_attn_dense_forward(const lsh_attn_desc *desc, const void *x, const void *v,
+                                  void *out, float *lse, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
+/* Workspace bytes lsh_attn_backward needs for `desc`. Writes *bytes. */
+lsh_status lsh_attn_backward_workspace_size(const lsh_attn_desc *desc, size_t *bytes);
+
+/* Gradients of lsh_attn_forward with respect to x and v, for training
+ * ("Reformer re-reading", §2.2, trains the model end to end). Bucket ids are
+ * an input, as in the forward they were computed from (the hash is piecewise
+ * constant and is not differentiated), and the sort is recomputed from them.
+ *   x, v [B][H][n][d]; buckets [B][H][Rn][n]; out [B][H][n][d] and lse
+ *   [B][H][Rn][n] from the forward on those inputs; dout = dL/dout
+ *   [B][H][n][d]; dlse = dL/dlse [B][H][Rn][n] fp32 or NULL (zero);
+ *   dx, dv [B][H][n][d] out. x, v, out, dout, dx, dv in desc.dtype.
+ * Supported: LSH_BF16 with chunk 64 and n % 64 == 0 (else
+ * LSH_ERR_UNSUPPORTED); other limits as for lsh_attn_forward.
+ * The gradient is that of the definition: the self logit and masked keys
+ * carry none, and the rounds' merge weights are differentiated; the round
+ * outputs themselves are not needed (their term cancels). Deterministic.
+ * Conventions (ownership, asynchrony, errors) as for lsh_attn_forward;
+ * bucket ids outside [0, nb) are clamped and reported as there. */
+lsh_status lsh_attn_backward(const lsh_attn_desc *desc, const void *x, const void *v,
+                             const int32_t *buckets, const void *out, const float *lse,
+                             const void *dout, const float *dlse, void *dx, void *dv,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
 /* Static, human-readable name of a status code. */
 const char *lsh_attn_status_string(lsh_status status);
 

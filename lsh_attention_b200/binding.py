@@ -25,7 +25,9 @@ _DTYPES = {torch.float32: LSH_F32, torch.bfloat16: LSH_BF16}
 #: every symbol the header declares
 EXPORTS = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_attn_forward",
            "lsh_attn_forward_profiled", "lsh_attn_get_device_status", "lsh_attn_get_diag",
-           "lsh_attn_sort_noalloc", "lsh_attn_selftest_wait_timeout", "lsh_attn_status_string")
+           "lsh_attn_sort_noalloc", "lsh_attn_selftest_wait_timeout",
+           "lsh_attn_dense_workspace_size", "lsh_attn_dense_forward",
+           "lsh_attn_backward_workspace_size", "lsh_attn_backward", "lsh_attn_status_string")
 
 
 class LshAttnDesc(ctypes.Structure):
@@ -73,6 +75,10 @@ def load() -> ctypes.CDLL:
             lib.lsh_attn_sort_noalloc.argtypes = [dp, vp, vp, vp]
             lib.lsh_attn_get_diag.argtypes = [vp, vp, ctypes.POINTER(LshAttnDiag)]
             lib.lsh_attn_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
+            lib.lsh_attn_dense_workspace_size.argtypes = [dp, ctypes.POINTER(sz)]
+            lib.lsh_attn_dense_forward.argtypes = [dp, vp, vp, vp, vp, vp, sz, vp]
+            lib.lsh_attn_backward_workspace_size.argtypes = [dp, ctypes.POINTER(sz)]
+            lib.lsh_attn_backward.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
             lib.lsh_attn_status_string.argtypes = [ctypes.c_int]
             lib.lsh_attn_status_string.restype = ctypes.c_char_p
             for f in EXPORTS[:-1]:
@@ -145,16 +151,7 @@ _ws_cache: dict = {}
 def workspace(desc: LshAttnDesc, device, stream=None) -> torch.Tensor:
     """A cached workspace of at least the size `desc` needs, one per
     (device, stream): calls that may run concurrently must not share one."""
-    need = lsh_attn_workspace_size(desc)
-    dev = torch.device(device)
-    s = stream if stream is not None else torch.cuda.current_stream(dev)
-    key = (dev.index, s.cuda_stream)
-    ws = _ws_cache.get(key)
-    if ws is None or ws.numel() < need:
-        _ws_cache.pop(key, None)
-        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-        _ws_cache[key] = ws
-    return ws
+    return _scratch(device, stream, lsh_attn_workspace_size(desc))
 
 
 def lsh_attn_hash(x, R, n_buckets: int, buckets=None, ws=None, stream=None):
@@ -243,6 +240,79 @@ def lsh_attn_forward(x, v, R=None, *, n_buckets: int, chunk: int, causal: bool, 
         ev = (ctypes.c_void_p * PROFILE_EVENTS)(*[e.cuda_event for e in events])
         _check(load().lsh_attn_forward_profiled(*args, ev))
     return out, lse
+
+
+def lsh_attn_dense_forward(x, v, *, causal: bool, out=None, lse=None, ws=None, stream=None):
+    """Dense shared-QK attention (the full-attention baseline) of x, v
+    [B, H, n, d] bf16. Returns (out [B, H, n, d], lse [B, H, n] fp32)."""
+    _on_current_device(stream, x=x, v=v, out=out, lse=lse, ws=ws)
+    B, H, n, d = x.shape
+    _require(x, "x", torch.bfloat16, None)
+    _require(v, "v", torch.bfloat16, tuple(x.shape))
+    desc = make_desc(B, H, n, d, 2, 1, 1, causal, x.dtype)
+    if out is None:
+        out = torch.empty_like(x)
+    if lse is None:
+        lse = torch.empty((B, H, n), dtype=torch.float32, device=x.device)
+    _require(out, "out", torch.bfloat16, tuple(x.shape))
+    _require(lse, "lse", torch.float32, (B, H, n))
+    need = ctypes.c_size_t(0)
+    _check(load().lsh_attn_dense_workspace_size(ctypes.byref(desc), ctypes.byref(need)))
+    if ws is None:
+        ws = _scratch(x.device, stream, need.value)
+    elif ws.numel() < need.value:
+        raise ValueError(f"ws: {need.value} bytes needed, {ws.numel()} given")
+    _check(load().lsh_attn_dense_forward(ctypes.byref(desc), _ptr(x), _ptr(v), _ptr(out),
+                                         _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return out, lse
+
+
+def lsh_attn_backward(x, v, buckets, out, lse, dout, *, n_buckets: int, chunk: int,
+                      causal: bool, dlse=None, dx=None, dv=None, ws=None, stream=None):
+    """Gradients (dx, dv) [B, H, n, d] of lsh_attn_forward(x, v, buckets=...)
+    for upstream dout [B, H, n, d] (and dlse [B, H, rounds, n], or None),
+    given that forward's out and lse."""
+    _on_current_device(stream, x=x, v=v, buckets=buckets, out=out, lse=lse, dout=dout, dlse=dlse,
+                       dx=dx, dv=dv, ws=ws)
+    B, H, n, d = x.shape
+    rounds = buckets.shape[2]
+    _require(x, "x", None, None)
+    for name, t in (("v", v), ("out", out), ("dout", dout)):
+        _require(t, name, x.dtype, tuple(x.shape))
+    _require(buckets, "buckets", torch.int32, (B, H, rounds, n))
+    _require(lse, "lse", torch.float32, (B, H, rounds, n))
+    if dlse is not None:
+        _require(dlse, "dlse", torch.float32, (B, H, rounds, n))
+    desc = make_desc(B, H, n, d, n_buckets, chunk, rounds, causal, x.dtype)
+    if dx is None:
+        dx = torch.empty_like(x)
+    if dv is None:
+        dv = torch.empty_like(x)
+    _require(dx, "dx", x.dtype, tuple(x.shape))
+    _require(dv, "dv", x.dtype, tuple(x.shape))
+    need = ctypes.c_size_t(0)
+    _check(load().lsh_attn_backward_workspace_size(ctypes.byref(desc), ctypes.byref(need)))
+    if ws is None:
+        ws = _scratch(x.device, stream, need.value)
+    elif ws.numel() < need.value:
+        raise ValueError(f"ws: {need.value} bytes needed, {ws.numel()} given")
+    _check(load().lsh_attn_backward(ctypes.byref(desc), _ptr(x), _ptr(v), _ptr(buckets),
+                                    _ptr(out), _ptr(lse), _ptr(dout), _ptr(dlse), _ptr(dx),
+                                    _ptr(dv), _ptr(ws), ws.numel(), _stream(stream)))
+    return dx, dv
+
+
+def _scratch(device, stream, need: int) -> torch.Tensor:
+    """The cached workspace of (device, stream), grown to `need` bytes."""
+    dev = torch.device(device)
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    key = (dev.index, s.cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        _ws_cache.pop(key, None)
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        _ws_cache[key] = ws
+    return ws
 
 
 def lsh_attn_sort_noalloc(buckets, n_buckets: int, perm=None, stream=None):

@@ -1,0 +1,597 @@
+// Backward pass of the LSH-attention forward (bf16, chunk 64), on the
+// 5th-generation tensor cores.
+//
+// The forward is "Reformer summary" (ttnews.xyz), §局部敏感哈希注意力 and
+// §多輪LSH哈希, with the logit of "Reformer: LSH attention and reversible
+// layers" (dtcms.com), §二.1; the pages train it end to end ("Reformer
+// re-reading" (2kiu.com), §2.2). Bucket ids are an input (the hash is
+// piecewise constant), so the sort is recomputed from them.
+//
+// Derivation (upstream g = dL/dout, optional dlse_in = dL/dlse): with
+// w_r = exp(lse_r - LSE) the merge weights and o_r each round's output,
+//   dL/do_r = w_r g,   dL/dlse_r = w_r g.(o_r - out) + dlse_in_r.
+// Per round, for query i and key j of its window, P_ij = exp(l_ij - lse_r,i),
+//   dS_ij = P_ij (dP_ij - D_i + dL/dlse_r,i),  dP_ij = w_i g_i . v_j,
+//   D_i = rowsum(P_i dP_i) = w_i g_i . o_r,i,
+// and D_i cancels against the w_i g_i . o_r,i inside dL/dlse_r,i:
+//   dS_ij = P_ij (w_i g_i . v_j + c_i),   c_i = dlse_in_r,i - w_i g_i . out_i,
+// so no round's output is needed. The self logit and masked keys carry no
+// gradient (dS = 0 there). With l_ij = x_i . x_j kinv_j / sqrt(d) and
+// kd_j = kinv_j / sqrt(d), dS'_ij = dS_ij kd_j:
+//   dx_i (query role)  = sum_j dS'_ij x_j
+//   G_j = sum_i dS'_ij x_i,   dx_j (key role) = G_j - x_j kinv_j^2 (x_j . G_j)
+//   dv_j = sum_i P_ij w_i g_i
+// and each position sums its query and key roles over the rounds.
+//
+// Kernels:
+//   k_bwd_prep_pos   per position: LSE over rounds and g . out
+//   k_bwd_prep_slot  per (round, slot): (position, lse log2(e), w, c) and the
+//                    key's (logit scale, kd, kinv)
+//   k_bwd_dq         query-stationary, a pair of chunks per unit (128 queries,
+//                    192 keys as in the forward): S = Q K^T and dPraw = G V^T
+//                    into TMEM, dS' written over S in bf16, dQ = dS' X_window
+//                    (A read from TMEM); dQ rows out, fp32, slot order
+//   k_bwd_dkv        key-stationary, a pair of chunks of keys per unit (128
+//                    keys, the 192 queries that see them, in two passes of 128
+//                    and 64): S^T = K Q^T and dPraw^T = V G^T into TMEM,
+//                    P w and dS' written over them in bf16, dV += (P w) G_q and
+//                    G += dS' X_q (A read from TMEM); after both passes the key
+//                    rows of dx and dv out, fp32, slot order
+//   k_bwd_unsort     per position: dx = sum_r (dQ + dXk)[inv_r], dv = sum_r dV[inv_r]
+// Each unit runs in phases separated by CTA barriers (loads, MMAs, the
+// elementwise step, MMAs, write-out); TMEM holds [0, 512) for one unit.
+#pragma once
+
+#include "attn_tc.cuh"
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace lsh {
+
+constexpr int kBwdWarps = 8;  // warps 0-3 own TMEM lane quadrants; all 8 load
+constexpr float kBwdLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// grid-stride over (bh, position); block 256, one warp per position.
+// lse [BH][R][n] (natural log), out, g [BH][n][D] in T; pos_tab [BH][n]
+// float2 (LSE, g . out).
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    k_bwd_prep_pos(const float* __restrict__ lse, const T* __restrict__ out,
+                   const T* __restrict__ g, float2* __restrict__ pos_tab, int n, int rounds,
+                   int64_t total) {
+  constexpr int PER = D / 32;
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < total;
+       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int64_t bh = r / n;
+    const int i = (int)(r - bh * n);
+    float dot = 0.f;
+#pragma unroll
+    for (int k = 0; k < PER; ++k)
+      dot = fmaf(Elem<T>::to_f(g[r * D + lane + 32 * k]), Elem<T>::to_f(out[r * D + lane + 32 * k]),
+                 dot);
+    dot = warp_sum(dot);
+    float mx = -INFINITY;
+    for (int q = lane; q < rounds; q += 32) mx = fmaxf(mx, lse[(bh * rounds + q) * n + i]);
+    mx = warp_max(mx);
+    float z = 0.f;
+    for (int q = lane; q < rounds; q += 32) z += expf(lse[(bh * rounds + q) * n + i] - mx);
+    z = warp_sum(z);
+    if (lane == 0) pos_tab[r] = make_float2(mx + logf(z), dot);
+  }
+}
+
+// grid-stride over (seg, slot). perm [S][n]; lse, dlse (nullable) [S][n] by
+// position; pinv [BH][n]; qtab [S][n] float4 (position bits, lse log2(e), w,
+// c); ktab [S][n] float4 (logit scale kinv log2(e) / sqrt(d), kd, kinv, 0).
+__global__ void __launch_bounds__(256)
+    k_bwd_prep_slot(const int32_t* __restrict__ perm, const float* __restrict__ lse,
+                    const float* __restrict__ dlse, const float2* __restrict__ pos_tab,
+                    const float* __restrict__ pinv, float4* __restrict__ qtab,
+                    float4* __restrict__ ktab, int n, int rounds, float inv_sqrt_d,
+                    int64_t total) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t seg = e / n;
+    const int64_t bh = seg / rounds;
+    const int pos = perm[e];
+    const int64_t at = seg * n + pos;
+    const float l = lse[at];
+    const float2 pt = pos_tab[bh * n + pos];
+    const float w = expf(l - pt.x);
+    const float c = (dlse ? dlse[at] : 0.f) - w * pt.y;
+    const float kinv = pinv[bh * n + pos];
+    qtab[e] = make_float4(__int_as_float(pos), l * kBwdLog2e, w, c);
+    ktab[e] = make_float4(kinv * inv_sqrt_d * kBwdLog2e, kinv * inv_sqrt_d, kinv, 0.f);
+  }
+}
+
+// ---------------------------------------------------------------------------
+struct BwdArgs {
+  const __nv_bfloat16* x;  // [BH][n][d] position order
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* g;  // dL/dout [BH][n][d]
+  const float4* qtab;      // [S][n] per slot (position, lse2, w, c)
+  const float4* ktab;      // [S][n] per slot (ks, kd, kinv, 0)
+  float* dq;               // k_bwd_dq: [S][n][d] query-role dx, slot order
+  float* dxk;              // k_bwd_dkv: [S][n][d] key-role dx, slot order
+  float* dv;               // k_bwd_dkv: [S][n][d] dv, slot order
+  WsHeader* hdr;
+  int n, rounds, pairs_per_seg;
+  int64_t units;           // BH * pairs_per_seg * rounds
+};
+
+constexpr int kNoPos = 0x7fffffff;
+
+// Copies `rows` rows of src (position order, row `pos(r)`) into a swizzled
+// K-major tile [KH][rows][128 B] by cp.async, all threads of the CTA; a row
+// whose position is kNoPos is zero-filled.
+template <int D, typename PosFn>
+__device__ __forceinline__ void bwd_load_rows(unsigned char* tile, int rows,
+                                              const __nv_bfloat16* src, PosFn pos) {
+  constexpr int CPR = D / 8;  // 16-byte pieces per row
+  const uint32_t box = (uint32_t)rows * 128;
+  for (int e = threadIdx.x; e < rows * CPR; e += blockDim.x) {
+    const int row = e / CPR, piece = e % CPR;
+    const int kh = piece >> 3, cc = piece & 7;
+    const int p = pos(row);
+    const bool valid = p != kNoPos;
+    const __nv_bfloat16* s = valid ? src + (int64_t)p * D + piece * 8 : src;
+    sm100::cp_async16_zfill(tile + kh * box + row * 128 + ((cc ^ (row & 7)) << 4), s, valid);
+  }
+}
+
+// (batch-head, segment, first chunk) of unit u (numbered (batch, head), pair, round)
+__device__ __forceinline__ void bwd_unit(const BwdArgs& a, int64_t u, int64_t& bh, int64_t& seg,
+                                         int& c0) {
+  const int64_t per_bh = (int64_t)a.pairs_per_seg * a.rounds;
+  bh = u / per_bh;
+  const int rem = (int)(u - bh * per_bh);
+  const int pair = rem / a.rounds;
+  seg = bh * a.rounds + (rem - pair * a.rounds);
+  c0 = 2 * pair;
+}
+
+template <int D>
+inline size_t bwd_dq_smem() {
+  constexpr size_t KH = D / 64;
+  return 1024 + KH * 192 * 128 /* x window */ + KH * 192 * 128 /* v window */ +
+         KH * 128 * 128 /* g queries */ + 192 * 16 /* key table */ + 128 * 16 /* query table */ +
+         256;
+}
+
+// Query-stationary: dQ of the 128 queries of a chunk pair.
+// TMEM: S [0, 192) (dS' bf16 over [0, 96)), dPraw [192, 384), dQ [384, 384 + d).
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdWarps * 32, 1) k_bwd_dq(BwdArgs a) {
+  using namespace sm100;
+  constexpr int KH = D / 64;
+  constexpr uint32_t XBOX = 192 * 128, GBOX = 128 * 128;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* xt = base;                 // [KH][192][128 B] key window (queries: rows 64..191)
+  unsigned char* vt = xt + KH * XBOX;       // [KH][192][128 B]
+  unsigned char* gt = vt + KH * XBOX;       // [KH][128][128 B] g rows of the queries
+  float4* kt = reinterpret_cast<float4*>(gt + KH * GBOX);  // [192] (ks, kd, kinv, pos bits)
+  float4* qt = kt + 192;                                   // [128] (pos, lse2, w, c)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qt + 128);
+  uint64_t* bar_sp = bars;      // S and dP MMAs done
+  uint64_t* bar_q = bars + 1;   // dQ MMA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* bad = reinterpret_cast<volatile int*>(bars + 3);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(bar_sp, 1);
+    mbar_init(bar_q, 1);
+    *bad = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_dp = tmem + 192, tm_dq = tmem + 384;
+
+  int it = 0;
+  for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x, ++it) {
+    int64_t bh, seg;
+    int c0;
+    bwd_unit(a, u, bh, seg, c0);
+    const int k0 = (c0 - 1) * kAttnM;  // first key slot (may be < 0)
+    const int64_t so = seg * a.n;
+    // ---- tables and rows
+    for (int j = tid; j < 192; j += blockDim.x) {
+      const int ks = k0 + j;
+      float4 t = make_float4(0.f, 0.f, 0.f, __int_as_float(kNoPos));
+      if (ks >= 0 && ks < a.n) {
+        const float4 k = a.ktab[so + ks];
+        t = make_float4(k.x, k.y, k.z, a.qtab[so + ks].x);
+      }
+      kt[j] = t;
+      if (j >= kAttnM) {
+        const int qs = k0 + j;
+        qt[j - kAttnM] = (qs < a.n) ? a.qtab[so + qs]
+                                    : make_float4(__int_as_float(kNoPos), 0.f, 0.f, 0.f);
+      }
+    }
+    __syncthreads();
+    const __nv_bfloat16* xb = a.x + bh * a.n * D;
+    bwd_load_rows<D>(xt, 192, xb, [&](int r) { return __float_as_int(kt[r].w); });
+    bwd_load_rows<D>(vt, 192, a.v + bh * a.n * D, [&](int r) { return __float_as_int(kt[r].w); });
+    bwd_load_rows<D>(gt, 128, a.g + bh * a.n * D, [&](int r) { return __float_as_int(qt[r].x); });
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- S = Q K^T, dPraw = G_q V^T
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t xa = smem_u32(xt), va = smem_u32(vt), ga = smem_u32(gt);
+      const uint32_t idesc = idesc_bf16_f32(128, 192);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int kh = kk >> 2, ks = kk & 3;
+        mma_bf16_ss(tmem, desc_kmajor_sw128(xa + kh * XBOX + kAttnM * 128 + ks * 32),
+                    desc_kmajor_sw128(xa + kh * XBOX + ks * 32), idesc, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int kh = kk >> 2, ks = kk & 3;
+        mma_bf16_ss(tm_dp, desc_kmajor_sw128(ga + kh * GBOX + ks * 32),
+                    desc_kmajor_sw128(va + kh * XBOX + ks * 32), idesc, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_sp);
+    }
+    // ---- dS' = P (w dPraw + c) kd, over the S columns in bf16
+    if (warp < 4) {
+      if (!mbar_wait(bar_sp, it & 1)) *bad = 1;
+      tc_fence_after();
+      const int row = warp * 32 + lane;
+      const uint32_t tl = (uint32_t)(warp * 32) << 16;
+      const float4 me = qt[row];
+      const int qpos = __float_as_int(me.x);
+      const float lse2 = me.y, w = me.z, c = me.w;
+      const int wlo = warp < 2 ? 0 : kAttnM;  // the row's window: keys [wlo, wlo + 128)
+#pragma unroll 1
+      for (int b = 0; b < 6; ++b) {
+        uint32_t sv[32], dv_[32];
+        tmem_ld32(tmem + tl + b * 32, sv);
+        tmem_ld32(tm_dp + tl + b * 32, dv_);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int cc = 0; cc < 32; cc += 2) {
+          float o2[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int j = b * 32 + cc + h;
+            const float4 k = kt[j];
+            const int kp = __float_as_int(k.w);
+            const bool in_window = j >= wlo && j < wlo + 128 && kp != kNoPos;
+            const bool live = in_window && kp != qpos && (!CAUSAL || kp < qpos);
+            const float p = ex2_approx(fmaf(__uint_as_float(sv[cc + h]), k.x, -lse2));
+            const float ds = p * fmaf(w, __uint_as_float(dv_[cc + h]), c) * k.y;
+            o2[h] = live ? ds : 0.f;
+          }
+          pk[cc >> 1] = pack_bf16x2(o2[0], o2[1]);
+        }
+        tmem_st16(tmem + tl + b * 16, pk);
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    // ---- dQ = dS' X_window (A from TMEM, B = x window MN-major)
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t xa = smem_u32(xt);
+      const uint32_t idesc = idesc_bf16_f32(128, D) | (1u << 16);
+#pragma unroll
+      for (int kk = 0; kk < 192 / 16; ++kk)
+        mma_bf16_ts(tm_dq, tmem + kk * 8, desc_mnmajor_sw128(xa + kk * 16 * 128, XBOX), idesc,
+                    kk > 0 ? 1u : 0u);
+      mma_commit(bar_q);
+    }
+    if (warp < 4) {
+      if (!mbar_wait(bar_q, it & 1)) *bad = 1;
+      tc_fence_after();
+      const int row = warp * 32 + lane;
+      const uint32_t tl = (uint32_t)(warp * 32) << 16;
+      const int qs = c0 * kAttnM + row;
+#pragma unroll
+      for (int b = 0; b < D / 32; ++b) {
+        uint32_t o[32];
+        tmem_ld32(tm_dq + tl + b * 32, o);
+        tmem_wait_ld();
+        if (qs < a.n) {
+          float4* dst = reinterpret_cast<float4*>(a.dq + (so + qs) * D + b * 32);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
+                                 __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // TMEM and the tiles are reused by the next unit
+    if (*bad) break;  // uniform: read after the barrier
+  }
+  if (tid == 0 && *bad) record_status(a.hdr, 5u /* LSH_ERR_TIMEOUT */);
+  __syncthreads();
+  if (warp == 0 && !*bad) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+inline size_t bwd_dkv_smem() {
+  constexpr size_t KH = D / 64;
+  return 1024 + KH * 192 * 128 /* x rows of the queries (keys: rows 0..127) */ +
+         KH * 128 * 128 /* v rows of the keys */ + KH * 192 * 128 /* g rows of the queries */ +
+         128 * 16 /* key table */ + 192 * 16 /* query table */ + 256;
+}
+
+// Key-stationary: dv and the key-role dx of the 128 keys of a chunk pair.
+// Keys: slots [64 c0, 64 c0 + 128); queries: slots [64 c0, 64 c0 + 192).
+// TMEM: S^T [0, 128) (P w bf16 over [0, 64)), dPraw^T [128, 256) (dS' bf16
+// over [128, 192)), dV [256, 256 + d), G [384, 384 + d).
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdWarps * 32, 1) k_bwd_dkv(BwdArgs a) {
+  using namespace sm100;
+  constexpr int KH = D / 64;
+  constexpr uint32_t XBOX = 192 * 128, VBOX = 128 * 128;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* xt = base;                 // [KH][192][128 B] x of the queries
+  unsigned char* vt = xt + KH * XBOX;       // [KH][128][128 B] v of the keys
+  unsigned char* gt = vt + KH * VBOX;       // [KH][192][128 B] g of the queries
+  float4* kt = reinterpret_cast<float4*>(gt + KH * XBOX);  // [128] (ks, kd, kinv, pos bits)
+  float4* qt = kt + 128;                                   // [192] (pos, lse2, w, c)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(qt + 192);
+  uint64_t* bar_sp = bars;     // S^T and dP^T MMAs of a pass done
+  uint64_t* bar_acc = bars + 1;  // dV and G MMAs of a pass done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* bad = reinterpret_cast<volatile int*>(bars + 3);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    mbar_init(bar_sp, 1);
+    mbar_init(bar_acc, 1);
+    *bad = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_dp = tmem + 128, tm_dv = tmem + 256, tm_g = tmem + 384;
+
+  int phase = 0;  // completions of each barrier so far (both complete twice per unit)
+  for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x) {
+    int64_t bh, seg;
+    int c0;
+    bwd_unit(a, u, bh, seg, c0);
+    const int s0 = c0 * kAttnM;  // first key slot and first query slot
+    const int64_t so = seg * a.n;
+    for (int j = tid; j < 192; j += blockDim.x) {
+      const int s = s0 + j;
+      const bool valid = s < a.n;
+      const float4 q = valid ? a.qtab[so + s] : make_float4(__int_as_float(kNoPos), 0.f, 0.f, 0.f);
+      qt[j] = q;
+      if (j < 128) {
+        const float4 k = valid ? a.ktab[so + s] : make_float4(0.f, 0.f, 0.f, 0.f);
+        kt[j] = make_float4(k.x, k.y, k.z, q.x);
+      }
+    }
+    __syncthreads();
+    const int64_t ho = bh * a.n * D;
+    bwd_load_rows<D>(xt, 192, a.x + ho, [&](int r) { return __float_as_int(qt[r].x); });
+    bwd_load_rows<D>(vt, 128, a.v + ho, [&](int r) { return __float_as_int(kt[r].w); });
+    bwd_load_rows<D>(gt, 192, a.g + ho, [&](int r) { return __float_as_int(qt[r].x); });
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    for (int pass = 0; pass < 2; ++pass, ++phase) {
+      const int q0 = pass * 128, N = pass == 0 ? 128 : 64;  // queries [q0, q0 + N)
+      // ---- S^T = K Q^T, dPraw^T = V_k G_q^T
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t xa = smem_u32(xt), va = smem_u32(vt), ga = smem_u32(gt);
+        const uint32_t idesc = idesc_bf16_f32(128, N);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int kh = kk >> 2, ks = kk & 3;
+          mma_bf16_ss(tmem, desc_kmajor_sw128(xa + kh * XBOX + ks * 32),
+                      desc_kmajor_sw128(xa + kh * XBOX + q0 * 128 + ks * 32), idesc,
+                      kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int kh = kk >> 2, ks = kk & 3;
+          mma_bf16_ss(tm_dp, desc_kmajor_sw128(va + kh * VBOX + ks * 32),
+                      desc_kmajor_sw128(ga + kh * XBOX + q0 * 128 + ks * 32), idesc,
+                      kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_sp);
+      }
+      // ---- P w and dS' for key row j (thread), queries [q0, q0 + N)
+      if (warp < 4) {
+        if (!mbar_wait(bar_sp, phase & 1)) *bad = 1;
+        tc_fence_after();
+        const int j = warp * 32 + lane;
+        const uint32_t tl = (uint32_t)(warp * 32) << 16;
+        const float4 k = kt[j];
+        const int kp = __float_as_int(k.w);
+        const int kc = j / kAttnM;  // key chunk within the unit (0 or 1)
+#pragma unroll 1
+        for (int b = 0; b < N / 32; ++b) {
+          uint32_t sv[32], dv_[32];
+          tmem_ld32(tmem + tl + b * 32, sv);
+          tmem_ld32(tm_dp + tl + b * 32, dv_);
+          tmem_wait_ld();
+          uint32_t pw[16], pd[16];
+#pragma unroll
+          for (int cc = 0; cc < 32; cc += 2) {
+            float ow[2], od[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int i = q0 + b * 32 + cc + h;  // query index in the unit
+              const float4 q = qt[i];
+              const int qp = __float_as_int(q.x);
+              const int qc = i / kAttnM;  // query chunk within the unit (0, 1 or 2)
+              // query chunk qc sees key chunks qc - 1 and qc
+              const bool window = kp != kNoPos && qp != kNoPos && (kc == qc || kc == qc - 1);
+              const bool self = window && kp == qp;
+              const bool live = window && kp != qp && (!CAUSAL || kp < qp);
+              // the self logit is -1e5: weight 1 for a row that sees only
+              // itself (its lse is -1e5), 0 otherwise; no gradient through it
+              const float l2 = self ? kSelfLogit * kBwdLog2e : __uint_as_float(sv[cc + h]) * k.x;
+              const float p = ex2_approx(l2 - q.y);
+              const float pv = (live || self) ? p : 0.f;
+              ow[h] = pv * q.z;
+              od[h] = live ? p * fmaf(q.z, __uint_as_float(dv_[cc + h]), q.w) * k.y : 0.f;
+            }
+            pw[cc >> 1] = pack_bf16x2(ow[0], ow[1]);
+            pd[cc >> 1] = pack_bf16x2(od[0], od[1]);
+          }
+          tmem_st16(tmem + tl + b * 16, pw);
+          tmem_st16(tm_dp + tl + b * 16, pd);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncthreads();
+      // ---- dV += (P w) G_q, G += dS' X_q (A from TMEM; B MN-major, K = queries)
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t xa = smem_u32(xt), ga = smem_u32(gt);
+        const uint32_t idesc = idesc_bf16_f32(128, D) | (1u << 16);
+        for (int kk = 0; kk < N / 16; ++kk) {
+          const uint32_t acc = (pass > 0 || kk > 0) ? 1u : 0u;
+          mma_bf16_ts(tm_dv, tmem + kk * 8, desc_mnmajor_sw128(ga + (q0 + kk * 16) * 128, XBOX),
+                      idesc, acc);
+          mma_bf16_ts(tm_g, tm_dp + kk * 8, desc_mnmajor_sw128(xa + (q0 + kk * 16) * 128, XBOX),
+                      idesc, acc);
+        }
+        mma_commit(bar_acc);
+      }
+      if (warp < 4) {
+        if (!mbar_wait(bar_acc, phase & 1)) *bad = 1;
+        tc_fence_after();
+      }
+      tc_fence_before();
+      __syncthreads();  // S^T / dP^T columns are rewritten by the next pass
+    }
+    // ---- key rows out: dv, and dx_key = G - x kinv^2 (x . G)
+    if (warp < 4) {
+      tc_fence_after();
+      const int j = warp * 32 + lane;
+      const uint32_t tl = (uint32_t)(warp * 32) << 16;
+      const int sj = s0 + j;
+      const float4 k = kt[j];
+      // the key's own x row is row j of the query tile (keys are its first
+      // 128 rows): 16-byte chunk c of each 64-column half at slot c ^ (j % 8)
+      auto xrow8 = [&](int e8, float (&f)[8]) {  // elements 8 e8 .. 8 e8 + 7
+        const unsigned char* line = xt + (e8 >> 3) * XBOX + j * 128;
+        Vec16<__nv_bfloat16>::unpack(
+            *reinterpret_cast<const uint4*>(line + (((e8 & 7) ^ (j & 7)) << 4)), f);
+      };
+      float xg = 0.f;
+#pragma unroll
+      for (int b = 0; b < D / 32; ++b) {
+        uint32_t gv[32];
+        tmem_ld32(tm_g + tl + b * 32, gv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float f[8];
+          xrow8(b * 4 + q, f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xg = fmaf(f[e], __uint_as_float(gv[8 * q + e]), xg);
+        }
+      }
+      const float fk = k.z * k.z * xg;
+#pragma unroll
+      for (int b = 0; b < D / 32; ++b) {
+        uint32_t gv[32], vv[32];
+        tmem_ld32(tm_g + tl + b * 32, gv);
+        tmem_ld32(tm_dv + tl + b * 32, vv);
+        tmem_wait_ld();
+        if (sj < a.n) {
+          float4* dx = reinterpret_cast<float4*>(a.dxk + (so + sj) * D + b * 32);
+          float4* dvv = reinterpret_cast<float4*>(a.dv + (so + sj) * D + b * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float f[8];
+            xrow8(b * 4 + q, f);
+            dx[2 * q] = make_float4(__uint_as_float(gv[8 * q]) - f[0] * fk,
+                                    __uint_as_float(gv[8 * q + 1]) - f[1] * fk,
+                                    __uint_as_float(gv[8 * q + 2]) - f[2] * fk,
+                                    __uint_as_float(gv[8 * q + 3]) - f[3] * fk);
+            dx[2 * q + 1] = make_float4(__uint_as_float(gv[8 * q + 4]) - f[4] * fk,
+                                        __uint_as_float(gv[8 * q + 5]) - f[5] * fk,
+                                        __uint_as_float(gv[8 * q + 6]) - f[6] * fk,
+                                        __uint_as_float(gv[8 * q + 7]) - f[7] * fk);
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dvv[q] = make_float4(__uint_as_float(vv[4 * q]), __uint_as_float(vv[4 * q + 1]),
+                                 __uint_as_float(vv[4 * q + 2]), __uint_as_float(vv[4 * q + 3]));
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*bad) break;
+  }
+  if (tid == 0 && *bad) record_status(a.hdr, 5u /* LSH_ERR_TIMEOUT */);
+  __syncthreads();
+  if (warp == 0 && !*bad) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// grid-stride over (bh, position), a warp per position (d / 32 elements per
+// lane): sums the query and key roles of every round through inv.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+    k_bwd_unsort(const int32_t* __restrict__ inv, const float* __restrict__ dq,
+                 const float* __restrict__ dxk, const float* __restrict__ dvs,
+                 T* __restrict__ dx, T* __restrict__ dv, int n, int rounds, int64_t total) {
+  constexpr int PER = D / 32;
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < total;
+       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    const int64_t bh = r / n;
+    const int i = (int)(r - bh * n);
+    float ax[PER], av[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) ax[k] = av[k] = 0.f;
+    for (int q = 0; q < rounds; ++q) {
+      const int64_t seg = bh * rounds + q;
+      const int64_t row = (seg * n + inv[seg * n + i]) * D;
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        ax[k] += dq[row + lane + 32 * k] + dxk[row + lane + 32 * k];
+        av[k] += dvs[row + lane + 32 * k];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+      dx[r * D + lane + 32 * k] = Elem<T>::from_f(ax[k]);
+      dv[r * D + lane + 32 * k] = Elem<T>::from_f(av[k]);
+    }
+  }
+}
+
+}  // namespace lsh

@@ -8,6 +8,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include "attn_dense.cuh"
+#include "bwd.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
@@ -452,6 +454,186 @@ lsh_status forward_typed(const Dims& D, const Layout& L, const void* x, const vo
   return mark(ev, 9, st);
 }
 
+// ---------------------------------------------------------------- dense
+struct DenseDims {
+  int n, d, causal, qtiles, kstride;
+  int64_t BH;
+  size_t kscale, queue, total;  // workspace layout
+};
+
+lsh_status check_dense(const lsh_attn_desc* desc, DenseDims* D) {
+  if (!desc) return LSH_ERR_INVALID_ARG;
+  const lsh_attn_desc& q = *desc;
+  if (q.batch < 1 || q.heads < 1 || q.n < 1 || q.d < 1 || (q.causal != 0 && q.causal != 1) ||
+      (q.dtype != LSH_F32 && q.dtype != LSH_BF16))
+    return LSH_ERR_INVALID_ARG;
+  if (q.dtype != LSH_BF16 || (q.d != 64 && q.d != 128)) return LSH_ERR_UNSUPPORTED;
+  D->n = q.n;
+  D->d = q.d;
+  D->causal = q.causal;
+  D->BH = (int64_t)q.batch * q.heads;
+  D->qtiles = (q.n + kDenseTile - 1) / kDenseTile;
+  D->kstride = D->qtiles * kDenseTile;
+  if (D->BH * D->kstride >= (int64_t(1) << 31)) return LSH_ERR_UNSUPPORTED;
+  if (D->BH > 65535) return LSH_ERR_UNSUPPORTED;  // TMA outer coordinate
+  size_t off = align_up(sizeof(WsHeader), 256);
+  D->kscale = off;
+  off = align_up(off + (size_t)D->BH * D->kstride * 4, 256);
+  D->queue = off;
+  off = align_up(off + (size_t)D->BH * q.n * 4, 256);
+  D->total = off;
+  return LSH_OK;
+}
+
+template <int DD, bool CAUSAL>
+lsh_status launch_dense(const DenseDims& D, const void* x, const void* v, void* out, float* lse,
+                        void* ws, cudaStream_t st) {
+  constexpr int NST = DD == 64 ? 4 : 2;  // K/V ring depth that fits shared memory
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  float* kscale = at<float>(ws, D.kscale);
+  int32_t* queue = at<int32_t>(ws, D.queue);
+  const int sms = sm_count();
+  {
+    const int64_t total = D.BH * D.kstride;
+    const int per_block = 256 / (DD / 8);
+    const unsigned blocks =
+        (unsigned)std::min<int64_t>((total + per_block - 1) / per_block, (int64_t)8 * sms);
+    k_dense_kscale<DD><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), kscale, D.n,
+                                               D.kstride, total);
+  }
+  CUtensorMap tmx, tmv, tmo;
+  if (!make_tmap_bf16_3d(&tmx, x, DD, D.n, D.BH, 64, kDenseTile) ||
+      !make_tmap_bf16_3d(&tmv, v, DD, D.n, D.BH, 64, kDenseTile) ||
+      !make_tmap_bf16_3d(&tmo, out, DD, D.n, D.BH, 64, 32))
+    return LSH_ERR_CUDA;
+  DenseArgs a;
+  a.kscale = kscale;
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.lse = lse;
+  a.fix_queue = queue;
+  a.hdr = hdr;
+  a.n = D.n;
+  a.BH = (int)D.BH;
+  a.qtiles = D.qtiles;
+  a.kstride = D.kstride;
+  a.units = D.BH * D.qtiles;
+  const unsigned grid = (unsigned)std::min<int64_t>(a.units, sms);
+  const size_t smem = dense_smem<DD, NST>();
+  auto kern = k_attn_dense<DD, CAUSAL, NST>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return LSH_ERR_CUDA;
+  kern<<<grid, kDenseWarps * 32, smem, st>>>(tmx, tmv, tmo, a);
+  // rows queued by the kernel (none for inputs of moderate norm) are redone exactly
+  k_dense_fixup<DD, CAUSAL><<<2 * sms, 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(v), kscale,
+      static_cast<__nv_bfloat16*>(out), lse, queue, hdr, D.n, D.kstride);
+  return last_cuda();
+}
+
+// ---------------------------------------------------------------- backward
+struct BwdLayout {
+  size_t header, perm, inv, hist, pinv, pos_tab, qtab, ktab, dq, dxk, dv, total;
+};
+
+// Backward support: bf16 and the tensor-core chunk (64), as the forward's
+// tensor-core path.
+lsh_status check_bwd(const lsh_attn_desc* desc, Dims* D, BwdLayout* L) {
+  lsh_status s = check_desc(desc, D, true);
+  if (s != LSH_OK) return s;
+  if (!attn_tc_supported(*D)) return LSH_ERR_UNSUPPORTED;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const size_t sn = (size_t)D->S * D->n;
+  L->header = take(sizeof(WsHeader));
+  L->perm = take(sn * 4);
+  L->inv = take(sn * 4);
+  L->hist = take((size_t)D->S * D->nb * D->tiles * 4);
+  L->pinv = take((size_t)D->BH * D->n * 4);
+  L->pos_tab = take((size_t)D->BH * D->n * 8);
+  L->qtab = take(sn * 16);
+  L->ktab = take(sn * 16);
+  L->dq = take(sn * D->d * 4);
+  L->dxk = take(sn * D->d * 4);
+  L->dv = take(sn * D->d * 4);
+  L->total = off;
+  return LSH_OK;
+}
+
+template <int DD, bool CAUSAL>
+lsh_status launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
+  const int sms = sm_count();
+  const unsigned grid = (unsigned)std::min<int64_t>(a.units, sms);
+  {
+    auto kern = k_bwd_dq<DD, CAUSAL>;
+    const size_t smem = bwd_dq_smem<DD>();
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, kBwdWarps * 32, smem, st>>>(a);
+  }
+  {
+    auto kern = k_bwd_dkv<DD, CAUSAL>;
+    const size_t smem = bwd_dkv_smem<DD>();
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return LSH_ERR_CUDA;
+    kern<<<grid, kBwdWarps * 32, smem, st>>>(a);
+  }
+  return last_cuda();
+}
+
+template <int DD>
+lsh_status backward_d(const Dims& D, const BwdLayout& L, const void* x, const void* v,
+                      const int32_t* buckets, const void* out, const float* lse,
+                      const void* dout, const float* dlse, void* dx, void* dv, void* ws,
+                      cudaStream_t st) {
+  using T = __nv_bfloat16;
+  WsHeader* hdr = at<WsHeader>(ws, L.header);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* inv = at<int32_t>(ws, L.inv);
+  lsh_status s = launch_sort<T>(D, buckets, x, v, perm, inv, nullptr, nullptr, nullptr,
+                                at<int32_t>(ws, L.hist), hdr, st);
+  if (s != LSH_OK) return s;
+  float* pinv = at<float>(ws, L.pinv);
+  if ((s = launch_row_invnorm(D, x, pinv, st)) != LSH_OK) return s;
+  const int sms = sm_count();
+  const int64_t pos_total = D.BH * D.n;
+  float2* pos_tab = at<float2>(ws, L.pos_tab);
+  k_bwd_prep_pos<T, DD><<<(unsigned)std::min<int64_t>((pos_total + 7) / 8, 8 * sms), 256, 0, st>>>(
+      lse, static_cast<const T*>(out), static_cast<const T*>(dout), pos_tab, D.n, D.rounds,
+      pos_total);
+  const int64_t slot_total = D.S * D.n;
+  float4* qtab = at<float4>(ws, L.qtab);
+  float4* ktab = at<float4>(ws, L.ktab);
+  k_bwd_prep_slot<<<(unsigned)std::min<int64_t>((slot_total + 255) / 256, 8 * sms), 256, 0, st>>>(
+      perm, lse, dlse, pos_tab, pinv, qtab, ktab, D.n, D.rounds, 1.0f / sqrtf((float)DD),
+      slot_total);
+  BwdArgs a;
+  a.x = static_cast<const T*>(x);
+  a.v = static_cast<const T*>(v);
+  a.g = static_cast<const T*>(dout);
+  a.qtab = qtab;
+  a.ktab = ktab;
+  a.dq = at<float>(ws, L.dq);
+  a.dxk = at<float>(ws, L.dxk);
+  a.dv = at<float>(ws, L.dv);
+  a.hdr = hdr;
+  a.n = D.n;
+  a.rounds = D.rounds;
+  a.pairs_per_seg = (D.n / kAttnM + 1) / 2;
+  a.units = D.S * a.pairs_per_seg;
+  if ((s = D.causal ? launch_bwd_tc<DD, true>(a, st) : launch_bwd_tc<DD, false>(a, st)) != LSH_OK)
+    return s;
+  k_bwd_unsort<T, DD><<<(unsigned)std::min<int64_t>((pos_total + 7) / 8, 8 * sms), 256, 0, st>>>(
+      inv, a.dq, a.dxk, a.dv, static_cast<T*>(dx), static_cast<T*>(dv), D.n, D.rounds, pos_total);
+  return last_cuda();
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ C ABI
@@ -543,6 +725,62 @@ lsh_status lsh_attn_forward_profiled(const lsh_attn_desc* desc, const void* x, c
   return D.dtype == LSH_BF16
              ? forward_typed<__nv_bfloat16>(D, L, x, v, R, buckets, out, lse, ws, st, events)
              : forward_typed<float>(D, L, x, v, R, buckets, out, lse, ws, st, events);
+}
+
+lsh_status lsh_attn_dense_workspace_size(const lsh_attn_desc* desc, size_t* bytes) {
+  DenseDims D;
+  lsh_status s = check_dense(desc, &D);
+  if (s != LSH_OK) return s;
+  if (!bytes) return LSH_ERR_INVALID_ARG;
+  *bytes = D.total;
+  return LSH_OK;
+}
+
+lsh_status lsh_attn_dense_forward(const lsh_attn_desc* desc, const void* x, const void* v,
+                                  void* out, float* lse, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  DenseDims D;
+  lsh_status s = check_dense(desc, &D);
+  if (s != LSH_OK) return s;
+  if (!x || !v || !out || !lse) return LSH_ERR_INVALID_ARG;
+  if (!(aligned16(x) && aligned16(v) && aligned16(out))) return LSH_ERR_INVALID_ARG;
+  if (!ws || ((uintptr_t)ws & 255) != 0 || ws_bytes < D.total) return LSH_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = reset_header(ws, st)) != LSH_OK) return s;
+  if (D.d == 64)
+    return D.causal ? launch_dense<64, true>(D, x, v, out, lse, ws, st)
+                    : launch_dense<64, false>(D, x, v, out, lse, ws, st);
+  return D.causal ? launch_dense<128, true>(D, x, v, out, lse, ws, st)
+                  : launch_dense<128, false>(D, x, v, out, lse, ws, st);
+}
+
+lsh_status lsh_attn_backward_workspace_size(const lsh_attn_desc* desc, size_t* bytes) {
+  Dims D;
+  BwdLayout L;
+  lsh_status s = check_bwd(desc, &D, &L);
+  if (s != LSH_OK) return s;
+  if (!bytes) return LSH_ERR_INVALID_ARG;
+  *bytes = L.total;
+  return LSH_OK;
+}
+
+lsh_status lsh_attn_backward(const lsh_attn_desc* desc, const void* x, const void* v,
+                             const int32_t* buckets, const void* out, const float* lse,
+                             const void* dout, const float* dlse, void* dx, void* dv, void* ws,
+                             size_t ws_bytes, void* stream) {
+  Dims D;
+  BwdLayout L;
+  lsh_status s = check_bwd(desc, &D, &L);
+  if (s != LSH_OK) return s;
+  if (!x || !v || !buckets || !out || !lse || !dout || !dx || !dv) return LSH_ERR_INVALID_ARG;
+  if (!(aligned16(x) && aligned16(v) && aligned16(out) && aligned16(dout) && aligned16(dx) &&
+        aligned16(dv)))
+    return LSH_ERR_INVALID_ARG;
+  if (!ws || ((uintptr_t)ws & 255) != 0 || ws_bytes < L.total) return LSH_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = reset_header(ws, st)) != LSH_OK) return s;
+  return D.d == 64 ? backward_d<64>(D, L, x, v, buckets, out, lse, dout, dlse, dx, dv, ws, st)
+                   : backward_d<128>(D, L, x, v, buckets, out, lse, dout, dlse, dx, dv, ws, st);
 }
 
 lsh_status lsh_attn_get_diag(const void* ws, void* stream, lsh_attn_diag* diag) {

@@ -206,3 +206,15 @@ def forward_sampled(x, v, buckets, n_buckets: int, chunk: int, causal: bool, pos
     if rc != 0:
         raise ValueError(f"oracle sampled forward failed ({rc})")
     return out, lse
+
+
+def dense_sampled(x, v, causal: bool, pos, nthreads: int = 0):
+    """Dense shared-QK attention at sampled positions: the forward pass with
+    one round and one chunk spanning the sequence (every key is in the
+    query's window whatever the bucket ids). Returns (out [B, H, npos, d],
+    lse [B, H, npos])."""
+    x = _f64(x)
+    B, H, n, d = x.shape
+    zeros = np.zeros((B, H, 1, n), np.int32)
+    out, lse = forward_sampled(x, v, zeros, 2, n, causal, pos, nthreads)
+    return out, lse[:, :, 0]

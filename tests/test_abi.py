@@ -130,3 +130,18 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(lb, "_lib", None)
     with pytest.raises(ImportError):
         lb.load()
+
+
+def test_dense_host_checks(lib):
+    sz = ctypes.c_size_t(0)
+    assert lib.lsh_attn_dense_workspace_size(ctypes.byref(desc(n=1000)), ctypes.byref(sz)) == 0
+    # header, key scales [B*H][roundup(n, 128)], fixup queue [B*H*n]
+    assert sz.value >= 256 + 8 * 1024 * 4 + 8 * 1000 * 4
+    assert lib.lsh_attn_dense_workspace_size(ctypes.byref(desc(dtype=lb.LSH_F32)),
+                                             ctypes.byref(sz)) == 2
+    assert lib.lsh_attn_dense_workspace_size(ctypes.byref(desc(d=96)), ctypes.byref(sz)) == 2
+    assert lib.lsh_attn_dense_workspace_size(ctypes.byref(desc(n=0)), ctypes.byref(sz)) == 1
+    # null pointers and a missing workspace are refused before any launch
+    p = ctypes.c_void_p(256)
+    assert lib.lsh_attn_dense_forward(ctypes.byref(desc()), None, p, p, p, p, 1 << 30, None) == 1
+    assert lib.lsh_attn_dense_forward(ctypes.byref(desc()), p, p, p, p, None, 0, None) == 3

@@ -384,3 +384,18 @@ def test_sampled_forward_matches_full():
     so, sl = oracle.forward_sampled(x, v, bk, nb, m, True, pos)
     np.testing.assert_array_equal(so, out[:, :, pos])
     np.testing.assert_array_equal(sl, lse[:, :, :, pos])
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_dense_sampled_is_textbook_dense_attention(causal):
+    """oracle.dense_sampled (the baseline's reference) against the textbook
+    dense attention written above, at every position of two heads."""
+    g = rng(31)
+    x = g.standard_normal((1, 2, 40, 8))
+    v = g.standard_normal((1, 2, 40, 8))
+    pos = np.arange(40, dtype=np.int32)
+    out, lse = oracle.dense_sampled(x, v, causal, pos)
+    for h in range(2):
+        o_ref, l_ref = dense_attention(x[0, h], v[0, h], causal)
+        np.testing.assert_allclose(out[0, h], o_ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[0, h], l_ref, rtol=0, atol=1e-10)
