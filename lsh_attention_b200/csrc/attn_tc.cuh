@@ -16,30 +16,27 @@
 // neighbouring units of one (batch, head), so every round reads that head's
 // rows while they sit in L2 and HBM delivers each row about once.
 //
-// One persistent CTA per SM, 13 warps:
-//   warps 0-1   x loaders: the window's positions (perm) and key norms
-//               (1/||x|| by position) of the next unit are loaded into
-//               registers while the current unit's rows are in flight, then
-//               written to a 4-deep ring of (logit scale, position) per key;
-//               every 16-byte piece of the 192 x rows goes by cp.async to its
-//               place in the 128-byte-swizzled K-major tile (a slot outside
-//               [0, n) reads as zero). When a thread's copies have landed it
-//               fences them for the async proxy (the tensor cores read shared
-//               memory through it) and arrives.
-//   warps 2-3   v loaders: the same for the v rows, at the positions of the
-//               ring, into the tile of the P.V product.
-//   warp 4      tcgen05.mma: S(u+1) = Q K^T into TMEM S[s], then O(u) = P V
+// One persistent CTA per SM, 10 warps:
+//   warp 0      producer: the window's positions (perm) and key norms
+//               (1/||x|| by position) are loaded into registers two and one
+//               units ahead, written to a 4-deep ring of (logit scale,
+//               position) per key, and the 192 x rows and then the 192 v rows
+//               are gathered by position with TMA (tile::gather4: four rows of
+//               128 bytes per instruction, landing in the 128-byte-swizzled
+//               K-major tile by their shared-memory address); a slot outside
+//               [0, n) reads as zero.
+//   warp 1      tcgen05.mma: S(u+1) = Q K^T into TMEM S[s], then O(u) = P V
 //               with P read from TMEM, so S of the next unit is ready when
 //               the softmax warps finish the current one. The x tile is free
 //               again as soon as S is computed (the ring keeps the metadata).
-//   warps 5-8   softmax, one query row per thread, one pass: logits in log2
+//   warps 2-5   softmax, one query row per thread, one pass: logits in log2
 //               units are bounded by ||q|| log2(e) / sqrt(d) (keys have unit
 //               length), which serves as the stabiliser, so every probability
 //               is exp2(l - bound) <= 1 and is written to TMEM (bf16, over the
 //               dead S columns) as soon as it is computed; the row sum goes to
 //               the epilogue. A row whose only visible key is itself (the -1e5
 //               self logit) is flagged: its output is v of the query itself.
-//   warps 9-12  epilogue: O from TMEM, divided by the row sum and packed to
+//   warps 6-9   epilogue: O from TMEM, divided by the row sum and packed to
 //               bf16 (the accumulator is released before the stores), staged
 //               per warp in a 4 KB swizzled buffer (32 rows x 64 columns) and
 //               written by TMA bulk stores (slot order); the softmax writes lse
@@ -56,7 +53,7 @@ namespace lsh {
 
 constexpr int kAttnM = 64;      // chunk length served by this kernel
 constexpr int kAttnKeys = 192;  // key window of a pair of chunks
-constexpr int kAttnWarps = 13;
+constexpr int kAttnWarps = 10;
 constexpr int kAttnStats = 4;   // row-sum slots between softmax and epilogue
 constexpr int kAttnRing = 4;    // metadata ring depth
 // Above this bound (log2 units) the stabiliser could push exp2 below the
@@ -64,8 +61,7 @@ constexpr int kAttnRing = 4;    // metadata ring depth
 constexpr float kAttnBoundMax = 60.f;
 
 struct AttnTcArgs {
-  const __nv_bfloat16* x;      // [BH][n][d] position order
-  const __nv_bfloat16* v;      // [BH][n][d] position order
+  const __nv_bfloat16* v;      // [BH][n][d] position order (rows that see only themselves)
   const float* pinv;           // [BH][n] 1/||x|| by position (0 for a zero row)
   const int32_t* perm;         // [S][n] position of each slot
   float* lse;                  // [S][n] each round's lse by position (the caller's output)
@@ -90,13 +86,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnWarps * 32, 1)
-    k_attn_tc(const __grid_constant__ CUtensorMap tmo, AttnTcArgs a) {
+    k_attn_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmv,
+              const __grid_constant__ CUtensorMap tmo, AttnTcArgs a) {
   using namespace sm100;
   constexpr int KH = D / 64;
   constexpr uint32_t BOX = kAttnKeys * 128;
   constexpr uint32_t TILE = KH * BOX;
-  constexpr int CPR = KH * 8;       // 16-byte pieces per row
-  constexpr int RSTEP = 64 / CPR;   // rows between a loader thread's pieces
+  constexpr int ROWS = kAttnKeys / 32;  // window rows per producer lane
   constexpr float kLog2e = 1.4426950408889634f;
   constexpr int kNoKey = 0x7fffffff;
   extern __shared__ unsigned char smem_raw[];
@@ -108,9 +104,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   float2* ktab = reinterpret_cast<float2*>(ostage + 4 * 32 * 128);    // [ring][192] (scale, pos)
   float* rstat = reinterpret_cast<float*>(ktab + kAttnRing * kAttnKeys);  // [4][128] 1/sum
   uint64_t* bars = reinterpret_cast<uint64_t*>(rstat + kAttnStats * 128);
-  uint64_t* xfull = bars + 0;    // [2] x rows landed (64 x-loader threads)
+  uint64_t* xfull = bars + 0;    // [2] x rows landed (tx)
   uint64_t* xfree = bars + 2;    // [2] S MMA done with the x tile
-  uint64_t* vfull = bars + 4;    // [2] v rows landed (64 v-loader threads)
+  uint64_t* vfull = bars + 4;    // [2] v rows landed (tx)
   uint64_t* vfree = bars + 6;    // [2] PV MMA done with the v tile
   uint64_t* sfull = bars + 8;    // [2] S MMA done
   uint64_t* pready = bars + 10;  // [2] P written (4 softmax warps)
@@ -118,8 +114,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   uint64_t* ofull = bars + 14;   // PV MMA done
   uint64_t* ofree = bars + 15;   // 4 epilogue warps done reading O
   uint64_t* statf = bars + 16;   // [4] row sums written (4 softmax warps)
-  uint64_t* mfull = bars + 20;   // [ring] metadata written (64 x-loader threads)
-  uint64_t* mfree = bars + 24;   // [ring] 4 softmax warps + 2 v-loader warps done with it
+  uint64_t* mfull = bars + 20;   // [ring] metadata written (32 producer lanes)
+  uint64_t* mfree = bars + 24;   // [ring] 4 softmax warps done with it
   uint64_t* drain = bars + 28;   // MMA issuer: every issued MMA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 29);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 30);
@@ -131,9 +127,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(xfull + i, 64);
+      mbar_init(xfull + i, 1);
       mbar_init(xfree + i, 1);
-      mbar_init(vfull + i, 64);
+      mbar_init(vfull + i, 1);
       mbar_init(vfree + i, 1);
       mbar_init(sfull + i, 1);
       mbar_init(pready + i, 4);
@@ -143,15 +139,15 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     mbar_init(ofree, 4);
     for (int i = 0; i < kAttnStats; ++i) mbar_init(statf + i, 4);
     for (int i = 0; i < kAttnRing; ++i) {
-      mbar_init(mfull + i, 64);
-      mbar_init(mfree + i, 4 + 2);
+      mbar_init(mfull + i, 32);
+      mbar_init(mfree + i, 4);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     *drain_fail = 0;
     fence_mbar_init();
   }
-  if (warp == 4) tmem_alloc(tmem_slot, 512);
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -174,77 +170,111 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     c0 = 2 * pair;
   };
 
-  if (warp < 4) {
-    // ------------------------------------------------------------ loaders
-    const bool xl = warp < 2;      // x loaders write the ring; v loaders read it
-    const int lt = tid & 63;       // rank among this loader pair of warps
-    const unsigned char* src0 = reinterpret_cast<const unsigned char*>(xl ? a.x : a.v);
-    unsigned char* tiles = xl ? xt : vt;
-    uint64_t* full = xl ? xfull : vfull;
-    uint64_t* tfree = xl ? xfree : vfree;
-    const int piece = lt % CPR;    // this thread's 16-byte piece of every row it copies
-    const int kh = piece >> 3, cc = piece & 7;
-    // x loaders: positions and logit scales of the next unit's window (rows
-    // lt, lt + 64, lt + 128), loaded a unit ahead
-    int pj[3];
-    float sj[3];
-    auto fetch = [&](int i) {
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&tmx);
+      prefetch_tensormap(&tmv);
+    }
+    const int oob = (int)(a.units / a.rounds / a.pairs_per_seg) * a.n;  // rows: a row past them
+    // positions (perm) of a unit's window rows lane + 32 t, and their logit
+    // scales (1/||x|| c); the loads are issued two units (perm) and one unit
+    // (norms) before the values are used
+    auto perm_of = [&](int i, int (&p)[ROWS]) {
       int64_t bh, seg;
       int c0;
       unit_of(i, bh, seg, c0);
       const int k0 = (c0 - 1) * kAttnM;
 #pragma unroll
-      for (int q = 0; q < 3; ++q) {
-        const int ks = k0 + lt + 64 * q;
-        pj[q] = (ks >= 0 && ks < a.n) ? __ldg(a.perm + seg * a.n + ks) : kNoKey;
+      for (int t = 0; t < ROWS; ++t) {
+        const int ks = k0 + lane + 32 * t;
+        p[t] = (i < nu && ks >= 0 && ks < a.n) ? __ldg(a.perm + seg * a.n + ks) : kNoKey;
       }
-#pragma unroll
-      for (int q = 0; q < 3; ++q)
-        sj[q] = pj[q] != kNoKey ? __ldg(a.pinv + bh * a.n + pj[q]) * c_scale : 0.f;
     };
-    if (xl) fetch(0);
+    auto scale_of = [&](int i, const int (&p)[ROWS], float (&sc)[ROWS]) {
+      int64_t bh = 0, seg;
+      int c0;
+      if (i < nu) unit_of(i, bh, seg, c0);
+#pragma unroll
+      for (int t = 0; t < ROWS; ++t)
+        sc[t] = p[t] != kNoKey ? __ldg(a.pinv + bh * a.n + p[t]) * c_scale : 0.f;
+    };
+    int p0[ROWS], p1[ROWS], p2[ROWS];
+    float s0[ROWS], s1[ROWS];
+    perm_of(0, p0);
+    perm_of(1, p1);
+    scale_of(0, p0, s0);
+    scale_of(1, p1, s1);
+    perm_of(2, p2);
+    int lastx[2] = {-1, -1}, lastv[2] = {-1, -1};
+    bool ok = true;
     for (int i = 0; i < nu; ++i) {
       const int s = i & 1, k = i >> 1, m = i & (kAttnRing - 1), km = i / kAttnRing;
-      bool got;
-      if (xl)  // ring slot m free (unit i - 4 done with it), x tile s free (S of unit i - 2)
-        got = (km == 0 || mbar_wait(mfree + m, (km - 1) & 1)) &&
-              (k == 0 || mbar_wait(tfree + s, (k - 1) & 1));
-      else     // ring slot m written for unit i, v tile s free (PV of unit i - 2)
-        got = mbar_wait(mfull + m, km & 1) && (k == 0 || mbar_wait(tfree + s, (k - 1) & 1));
-      if (!got) fail();
-      // both warps of the pair stop together (a failure anywhere sets abort_flag)
-      if (bar_sync_any(2 + (xl ? 0 : 1), 64, !got || *abort_flag)) break;
-      float2* kt = ktab + m * kAttnKeys;
-      if (xl) {
-#pragma unroll
-        for (int q = 0; q < 3; ++q) kt[lt + 64 * q] = make_float2(sj[q], __int_as_float(pj[q]));
-        bar_sync_any(2, 64, false);  // the pair's ring entries are written
-        mbar_arrive(mfull + m);
+      // ring slot m free (the softmax of unit i - 4 is done with it), x tile s
+      // free (S of unit i - 2 computed)
+      bool got = (km == 0 || mbar_wait(mfree + m, (km - 1) & 1)) &&
+                 (k == 0 || mbar_wait(xfree + s, (k - 1) & 1));
+      if (__any_sync(0xffffffffu, !got || *abort_flag)) {
+        ok = __all_sync(0xffffffffu, got);
+        break;
       }
       int64_t bh, seg;
       int c0;
       unit_of(i, bh, seg, c0);
-      const unsigned char* rows = src0 + (bh * a.n) * (int64_t)(D * 2) + piece * 16;
-      unsigned char* dst = tiles + s * TILE + kh * BOX;
-#pragma unroll 4
-      for (int row = lt / CPR; row < kAttnKeys; row += RSTEP) {
-        const int pos = __float_as_int(kt[row].y);
-        const bool valid = pos != kNoKey;
-        const unsigned char* src = valid ? rows + (int64_t)pos * (D * 2) : src0;
-        cp_async16_zfill(dst + row * 128 + ((cc ^ (row & 7)) << 4), src, valid);
+      float2* kt = ktab + m * kAttnKeys;
+#pragma unroll
+      for (int t = 0; t < ROWS; ++t) kt[lane + 32 * t] = make_float2(s0[t], __int_as_float(p0[t]));
+      mbar_arrive(mfull + m);
+      __syncwarp();  // the ring is read back below by other lanes
+      const int rbase = (int)(bh * a.n);
+      // rows 4 g .. 4 g + 3 of the window, for g = lane and lane + 32 (< 48)
+      auto gather = [&](const CUtensorMap* map, unsigned char* tile, uint64_t* bar) {
+        for (int g = lane; g < kAttnKeys / 4; g += 32) {
+          int r[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int pos = __float_as_int(kt[4 * g + j].y);
+            r[j] = pos == kNoKey ? oob : rbase + pos;
+          }
+#pragma unroll
+          for (int kh = 0; kh < KH; ++kh)
+            tma_gather4_2d(tile + kh * BOX + 4 * g * 128, map, bar, kh * 64, r[0], r[1], r[2], r[3]);
+        }
+      };
+      if (lane == 0) mbar_expect_tx(xfull + s, TILE);
+      __syncwarp();
+      gather(&tmx, xt + s * TILE, xfull + s);
+      if (lane == 0) lastx[s] = k;
+      // the next units' metadata: norms one unit ahead, positions two
+#pragma unroll
+      for (int t = 0; t < ROWS; ++t) {
+        p0[t] = p1[t];
+        s0[t] = s1[t];
+        p1[t] = p2[t];
       }
-      cp_async_commit();
-      if (!xl) {  // done reading the ring slot
-        __syncwarp();
-        if (lane == 0) mbar_arrive(mfree + m);
+      scale_of(i + 1, p1, s1);
+      perm_of(i + 3, p2);
+      // v tile s free (PV of unit i - 2 done)
+      got = k == 0 || mbar_wait(vfree + s, (k - 1) & 1);
+      if (__any_sync(0xffffffffu, !got || *abort_flag)) {
+        ok = __all_sync(0xffffffffu, got);
+        break;
       }
-      if (xl && i + 1 < nu) fetch(i + 1);  // in flight while this unit's rows land
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(full + s);
+      if (lane == 0) mbar_expect_tx(vfull + s, TILE);
+      __syncwarp();
+      gather(&tmv, vt + s * TILE, vfull + s);
+      if (lane == 0) lastv[s] = k;
     }
-    cp_async_wait_all();  // nothing of this thread's still writes shared memory at exit
-  } else if (warp == 4) {
+    if (lane == 0) {
+      if (!ok) fail();
+      // No copy may still be writing this CTA's shared memory when it exits:
+      // wait (bounded) for the last phase issued on every stage.
+      for (int s = 0; s < 2; ++s)
+        if ((lastx[s] >= 0 && !mbar_wait(xfull + s, lastx[s] & 1)) ||
+            (lastv[s] >= 0 && !mbar_wait(vfull + s, lastv[s] & 1)))
+          *drain_fail = 1;
+    }
+  } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, kAttnKeys);
@@ -291,7 +321,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       mma_commit(drain);
       if (!mbar_wait(drain, 0)) *drain_fail = 1;
     }
-  } else if (warp < 9) {
+  } else if (warp < 6) {
     // ------------------------------------------------------------ softmax
     const int q = warp & 3;       // TMEM lane quadrant
     const int row = q * 32 + lane;
@@ -429,7 +459,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         if (inv <= 0.f)  // only the token itself is visible: its own value row
           vr = reinterpret_cast<const uint4*>(
               a.v + (bh * a.n + a.perm[seg * a.n + qs0 + lane]) * (int64_t)D);
-        unsigned char* stg = ostage + (warp - 9) * 32 * 128;
+        unsigned char* stg = ostage + (warp - 6) * 32 * 128;
 #pragma unroll
         for (int b = 0; b < D / 64; ++b) {  // 64 columns (128 bytes of bf16) per store
           if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
@@ -459,7 +489,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   __syncthreads();
   // after a drain that gave up, TMEM is left allocated rather than freed
   // under a running MMA; the status word already records the timeout
-  if (warp == 4 && !*drain_fail) {
+  if (warp == 1 && !*drain_fail) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -472,30 +502,42 @@ inline size_t attn_tc_smem(int D) {
 }
 
 // 1/||x|| of every row of x [rows][D] (bf16), for the attention's key scales
-// when the hash did not produce them: a group of D / 8 lanes per row, one
-// 16-byte piece per lane, the square sum reduced inside the group.
+// when the hash did not produce them. The square sum is formed in the order
+// the tensor-core hash's epilogue forms it (partial sums over the row's
+// 16-byte pieces p = r, r + P, r + 2P, ... for r < P = kNormParts, each
+// piece's elements in order, then 0 + part_0 + part_1 + ...), so both
+// sources give the same bits: a forward gets the same output whether the
+// hash runs inside it or the caller passes its bucket ids. A group of
+// kNormParts lanes per row.
 template <int D>
 __global__ void __launch_bounds__(256)
     k_row_invnorm(const __nv_bfloat16* __restrict__ x, float* __restrict__ pinv, int64_t rows) {
-  constexpr int L = D / 8;  // lanes per row: 8 or 16
+  constexpr int L = kNormParts;
+  constexpr int PIECES = D / 8;
   const int gl = threadIdx.x % L;
   const int64_t stride = (int64_t)gridDim.x * (blockDim.x / L);
-  // the same trip count for every lane of a warp (the group shuffles below)
-  const int64_t first = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / L;
-  const int64_t warp_first = first - (threadIdx.x & 31) / L;
+  const int64_t warp_first = ((int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31)) / L;
   for (int64_t r0 = warp_first; r0 < rows; r0 += stride) {
     const int64_t r = r0 + (threadIdx.x & 31) / L;
     float ss = 0.f;
     if (r < rows) {
-      const uint4 u = *reinterpret_cast<const uint4*>(x + r * D + gl * 8);
-      float f[8];
-      Vec16<__nv_bfloat16>::unpack(u, f);
+      const uint4* row = reinterpret_cast<const uint4*>(x + r * D);
+      uint4 u[PIECES / L];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+      for (int k = 0; k < PIECES / L; ++k) u[k] = row[gl + k * L];
+#pragma unroll
+      for (int k = 0; k < PIECES / L; ++k) {
+        float f[8];
+        Vec16<__nv_bfloat16>::unpack(u[k], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+      }
     }
+    // 0 + part_0 + part_1 + ..., in that order
+    float sst = 0.f;
 #pragma unroll
-    for (int o = L / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (r < rows && gl == 0) pinv[r] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+    for (int o = 0; o < L; ++o) sst += __shfl_sync(0xffffffffu, ss, (threadIdx.x & 31) - gl + o);
+    if (r < rows && gl == 0) pinv[r] = sst > 0.f ? 1.0f / sqrtf(sst) : 0.f;
   }
 }
 

@@ -8,6 +8,9 @@
 namespace lsh {
 
 constexpr float kSelfLogit = -1.0e5f;  // logit of a token against itself
+// ||x||^2 is summed in this many interleaved partial sums over a row's 16-byte
+// pieces, by the tensor-core hash and by the attention's norm pass alike
+constexpr int kNormParts = 2;
 
 // Workspace header: status word and counters, 256 bytes at the start of the
 // caller's workspace. Field order matches lsh_attn_diag.

@@ -35,6 +35,8 @@ constexpr int kHashEpiPerQuad = 3;   // epilogue warps per TMEM lane quadrant
 constexpr int kHashMaxBatches = 4;   // 16-column batches per epilogue warp and unit
 constexpr int kHashMaxN = 16 * kHashMaxBatches * kHashEpiPerQuad;  // columns per MMA (N): 192
 constexpr int kHashWarps = 2 + 4 * kHashEpiPerQuad;  // 0: TMA, 1: MMA, rest: epilogue
+// the norm pass of the attention forms ||x||^2 in this epilogue's order
+static_assert(kHashEpiPerQuad - 1 == kNormParts, "norm summation orders must agree");
 constexpr float kTieFactor = 4.0f;   // margin threshold / accumulation error bound
 constexpr int kHashSmemBudget = 227 * 1024;
 

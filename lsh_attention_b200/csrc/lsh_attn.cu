@@ -341,13 +341,14 @@ lsh_status launch_attn_simt(const Dims& D, const void* xs, const void* vs, const
 }
 
 template <int DD, bool CAUSAL>
-lsh_status launch_attn_tc_k(const CUtensorMap& tmo, const AttnTcArgs& a, unsigned grid,
+lsh_status launch_attn_tc_k(const CUtensorMap& tmx, const CUtensorMap& tmv,
+                            const CUtensorMap& tmo, const AttnTcArgs& a, unsigned grid,
                             size_t smem, cudaStream_t st) {
   auto kern = k_attn_tc<DD, CAUSAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return LSH_ERR_CUDA;
-  kern<<<grid, kAttnWarps * 32, smem, st>>>(tmo, a);
+  kern<<<grid, kAttnWarps * 32, smem, st>>>(tmx, tmv, tmo, a);
   return last_cuda();
 }
 
@@ -355,11 +356,15 @@ lsh_status launch_attn_tc_k(const CUtensorMap& tmo, const AttnTcArgs& a, unsigne
 lsh_status launch_attn_tc(const Dims& D, const void* x, const void* v, const int32_t* perm,
                           const float* pinv, void* out_r, float* lse, WsHeader* hdr,
                           cudaStream_t st) {
-  CUtensorMap tmo;
+  CUtensorMap tmx, tmv, tmo;
   const uint64_t rows = (uint64_t)D.S * D.n;
-  if (!make_tmap_bf16_2d(&tmo, out_r, D.d, rows, (uint64_t)D.d * 2, 64, 32)) return LSH_ERR_CUDA;
+  const uint64_t prow = (uint64_t)D.BH * D.n;  // rows of x and v (position order)
+  // x and v: one-row boxes for the gathers; each round's output: 32-row stores
+  if (!make_tmap_bf16_2d(&tmx, x, D.d, prow, (uint64_t)D.d * 2, 64, 1) ||
+      !make_tmap_bf16_2d(&tmv, v, D.d, prow, (uint64_t)D.d * 2, 64, 1) ||
+      !make_tmap_bf16_2d(&tmo, out_r, D.d, rows, (uint64_t)D.d * 2, 64, 32))
+    return LSH_ERR_CUDA;
   AttnTcArgs a;
-  a.x = static_cast<const __nv_bfloat16*>(x);
   a.v = static_cast<const __nv_bfloat16*>(v);
   a.pinv = pinv;
   a.perm = perm;
@@ -372,16 +377,16 @@ lsh_status launch_attn_tc(const Dims& D, const void* x, const void* v, const int
   const unsigned grid = (unsigned)std::min<int64_t>(a.units, sm_count());
   const size_t smem = attn_tc_smem(D.d);
   if (D.d == 64)
-    return D.causal ? launch_attn_tc_k<64, true>(tmo, a, grid, smem, st)
-                    : launch_attn_tc_k<64, false>(tmo, a, grid, smem, st);
-  return D.causal ? launch_attn_tc_k<128, true>(tmo, a, grid, smem, st)
-                  : launch_attn_tc_k<128, false>(tmo, a, grid, smem, st);
+    return D.causal ? launch_attn_tc_k<64, true>(tmx, tmv, tmo, a, grid, smem, st)
+                    : launch_attn_tc_k<64, false>(tmx, tmv, tmo, a, grid, smem, st);
+  return D.causal ? launch_attn_tc_k<128, true>(tmx, tmv, tmo, a, grid, smem, st)
+                  : launch_attn_tc_k<128, false>(tmx, tmv, tmo, a, grid, smem, st);
 }
 
 // 1/||x|| by position, when the hash has not written it.
 lsh_status launch_row_invnorm(const Dims& D, const void* x, float* pinv, cudaStream_t st) {
   const int64_t rows = D.BH * D.n;
-  const int per_block = 256 / (D.d / 8);
+  const int per_block = 256 / kNormParts;
   const unsigned blocks =
       (unsigned)std::min<int64_t>((rows + per_block - 1) / per_block, (int64_t)8 * sm_count());
   if (D.d == 64)

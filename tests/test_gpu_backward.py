@@ -80,7 +80,7 @@ def test_backward_self_only_rows():
 
 
 def test_backward_deterministic():
-    w = I.Workload("det-bwd", 1, 4, 2048, 128, 32, 2, True, "bf16")
+    w = I.Workload("det-bwd", 1, 4, 2048, 128, 32, 64, 2, True, "bf16")
     x, v = I.make_qkv(w)
     bk = I.make_buckets(w).cuda()
     xg, vg = x.cuda(), v.cuda()
