@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         s0[t] = s1[t];
         p1[t] = p2[t];
       }
-      scale_of(i + 1, p1, s1);
+      scale_of(i + 2, p1, s1);  // p1 now holds unit i + 2's positions
       perm_of(i + 3, p2);
       // v tile s free (PV of unit i - 2 done)
       got = k == 0 || mbar_wait(vfree + s, (k - 1) & 1);

@@ -176,19 +176,17 @@ def test_forward_internal_hash(w):
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
 
 
-@pytest.mark.parametrize("w,heads", [(I.LONG_64K, [0, 5]), (I.IMAGE_12K, [0, 7])] +
-                         [(s, [0, 7]) for s in SWEEP_LARGE],
-                         ids=lambda p: p.name if hasattr(p, "name") else str(p))
-def test_forward_timed_path(w, heads):
+@pytest.mark.parametrize("w", [I.LONG_64K, I.IMAGE_12K] + SWEEP_LARGE, ids=lambda w: w.name)
+def test_forward_timed_path(w):
     """The bench's call at full size: lsh_attn_forward(x, v, R, buckets=NULL),
-    where the tensor-core hash also counts the sort's histograms and the fp64
-    re-decision corrects them.
-      1. On the sampled heads the GPU's bucket ids (every round, every
-         position) equal the oracle's hash bit for bit.
-      2. The timed call's out and lse equal, bit for bit over every head, the
-         GPU forward fed those bucket ids (the separate histogram pass), so the
+    where the tensor-core hash also counts the sort's histograms and writes
+    the key norms.
+      1. The GPU's bucket ids (every batch, head, round and position) equal the
+         oracle's hash bit for bit.
+      2. The timed call's out and lse equal, bit for bit, the GPU forward fed
+         those bucket ids (histograms and norms from their own passes), so the
          fused histograms give the same permutation.
-      3. At sampled positions of the sampled heads, out and lse match the
+      3. At sampled positions of every (batch, head), out and lse match the
          oracle's forward on the oracle's own ids."""
     x, v = I.make_qkv(w)
     R = I.make_rotations(w)
@@ -201,18 +199,14 @@ def test_forward_timed_path(w, heads):
     assert torch.equal(out, out2) and torch.equal(lse, lse2), \
         "the fused-histogram forward differs from the caller-bucket forward"
     gbk = gbk.cpu().numpy()
+    ref_bk, _ = oracle.hash_all(x, R)
+    np.testing.assert_array_equal(gbk, ref_bk, err_msg=f"{w.name}: bucket ids")
     out = out.float().cpu().numpy()
     lse = lse.cpu().numpy()
     pos = sample_positions(w.n)
-    bsel = [0] if w.batch * w.n > 65536 else list(range(w.batch))
-    for h in heads:
-        xs, vs = x[bsel][:, h:h + 1], v[bsel][:, h:h + 1]
-        ref_bk, _ = oracle.hash_all(xs, R)
-        np.testing.assert_array_equal(gbk[bsel][:, h:h + 1], ref_bk,
-                                      err_msg=f"{w.name} h{h}: bucket ids")
-        ro, rl = oracle.forward_sampled(xs, vs, ref_bk, w.n_buckets, w.chunk, w.causal, pos)
-        check_close(out[bsel][:, h:h + 1][:, :, pos], ro, w.dtype, f"{w.name} h{h} out")
-        check_close(lse[bsel][:, h:h + 1][:, :, :, pos], rl, w.dtype, f"{w.name} h{h} lse")
+    ro, rl = oracle.forward_sampled(x, v, ref_bk, w.n_buckets, w.chunk, w.causal, pos)
+    check_close(out[:, :, pos], ro, w.dtype, f"{w.name} out")
+    check_close(lse[:, :, :, pos], rl, w.dtype, f"{w.name} lse")
 
 
 def test_forward_tie_moves_histogram_count():
