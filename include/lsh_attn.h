@@ -233,6 +233,52 @@ lsh_status lsh_attn_backward(const lsh_attn_desc *desc, const void *x, const voi
                              const void *dout, const float *dlse, void *dx, void *dv,
                              void *workspace, size_t workspace_bytes, void *stream);
 
+/* A reversible layer around the attention ("Reformer: LSH attention and
+ * reversible layers", §二.2 reversible residual and §二.3 chunked
+ * feed-forward): with x = [x1, x2],
+ *   y1 = x1 + Attn(x2),   y2 = x2 + FFN(y1),
+ * and back:  x2 = y2 - FFN(y1),   x1 = y1 - Attn(x2).
+ * Attn(x) = W_o applied to the heads of lsh_attn_forward(x W_qk^T, x W_v^T)
+ * (shared QK, d_model = heads * d_head), FFN(y) = max(y W1^T + b1, 0) W2^T
+ * + b2 computed ffn_chunk rows at a time (the rows are independent, so the
+ * chunk only bounds the intermediate buffer). */
+typedef struct {
+    int32_t batch, n;        /* sequences and their length (n % 128 == 0) */
+    int32_t d_model;         /* = heads * d_head, a multiple of 128 */
+    int32_t heads, d_head;   /* d_head in {64, 128} */
+    int32_t d_ff;            /* feed-forward width, a multiple of 128 */
+    int32_t ffn_chunk;       /* rows per feed-forward chunk, a multiple of 128 */
+    int32_t n_buckets, chunk, rounds, causal;  /* the attention's (chunk 64) */
+    int32_t hash_buckets;    /* forward: 1 = hash into `buckets`, 0 = read them */
+} lsh_rev_desc;
+
+/* Weights, bf16 stored out x in (row j holds output feature j), biases fp32
+ * (either may be NULL for zero). */
+typedef struct {
+    const void *w_qk, *w_v, *w_o;  /* [d_model][d_model] */
+    const void *w1;                /* [d_ff][d_model] */
+    const float *b1;               /* [d_ff] */
+    const void *w2;                /* [d_model][d_ff] */
+    const float *b2;               /* [d_model] */
+} lsh_rev_weights;
+
+/* Workspace bytes lsh_rev_block needs for `desc`. */
+lsh_status lsh_rev_workspace_size(const lsh_rev_desc *desc, size_t *bytes);
+
+/* inverse = 0: (in1, in2) = (x1, x2) -> (out1, out2) = (y1, y2); the bucket
+ * ids [batch][heads][rounds][n] are hashed from x2 W_qk^T under R into
+ * `buckets` (desc.hash_buckets = 1) or read from it (0).
+ * inverse = 1: (in1, in2) = (y1, y2) -> (out1, out2) = (x1, x2) with the
+ * forward's bucket ids read from `buckets` (R unused).
+ * All activations [batch][n][d_model] bf16, device memory, 16-byte aligned.
+ * Kernel status (the products' and the attention's) is read with
+ * lsh_attn_get_device_status(workspace). Other conventions as for
+ * lsh_attn_forward. */
+lsh_status lsh_rev_block(const lsh_rev_desc *desc, int inverse, const void *in1, const void *in2,
+                         const lsh_rev_weights *weights, const void *R, int32_t *buckets,
+                         void *out1, void *out2, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
 /* Static, human-readable name of a status code. */
 const char *lsh_attn_status_string(lsh_status status);
 

@@ -27,7 +27,8 @@ EXPORTS = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_att
            "lsh_attn_forward_profiled", "lsh_attn_get_device_status", "lsh_attn_get_diag",
            "lsh_attn_sort_noalloc", "lsh_attn_selftest_wait_timeout",
            "lsh_attn_dense_workspace_size", "lsh_attn_dense_forward",
-           "lsh_attn_backward_workspace_size", "lsh_attn_backward", "lsh_attn_status_string")
+           "lsh_attn_backward_workspace_size", "lsh_attn_backward", "lsh_rev_workspace_size",
+           "lsh_rev_block", "lsh_attn_status_string")
 
 
 class LshAttnDesc(ctypes.Structure):
@@ -38,6 +39,16 @@ class LshAttnDesc(ctypes.Structure):
 class LshAttnDiag(ctypes.Structure):
     _fields_ = [(k, ctypes.c_uint32) for k in
                 ("status", "hash_refined", "bad_bucket_ids", "reserved")]
+
+
+class LshRevDesc(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_int32) for k in
+                ("batch", "n", "d_model", "heads", "d_head", "d_ff", "ffn_chunk", "n_buckets",
+                 "chunk", "rounds", "causal", "hash_buckets")]
+
+
+class LshRevWeights(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in ("w_qk", "w_v", "w_o", "w1", "b1", "w2", "b2")]
 
 
 class LshAttnError(RuntimeError):
@@ -79,6 +90,11 @@ def load() -> ctypes.CDLL:
             lib.lsh_attn_dense_forward.argtypes = [dp, vp, vp, vp, vp, vp, sz, vp]
             lib.lsh_attn_backward_workspace_size.argtypes = [dp, ctypes.POINTER(sz)]
             lib.lsh_attn_backward.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+            lib.lsh_rev_workspace_size.argtypes = [ctypes.POINTER(LshRevDesc),
+                                                   ctypes.POINTER(sz)]
+            lib.lsh_rev_block.argtypes = [ctypes.POINTER(LshRevDesc), ctypes.c_int, vp, vp,
+                                          ctypes.POINTER(LshRevWeights), vp, vp, vp, vp, vp, sz,
+                                          vp]
             lib.lsh_attn_status_string.argtypes = [ctypes.c_int]
             lib.lsh_attn_status_string.restype = ctypes.c_char_p
             for f in EXPORTS[:-1]:
@@ -300,6 +316,58 @@ def lsh_attn_backward(x, v, buckets, out, lse, dout, *, n_buckets: int, chunk: i
                                     _ptr(out), _ptr(lse), _ptr(dout), _ptr(dlse), _ptr(dx),
                                     _ptr(dv), _ptr(ws), ws.numel(), _stream(stream)))
     return dx, dv
+
+
+def lsh_rev_block(in1, in2, weights: dict, *, heads: int, n_buckets: int, rounds: int,
+                  causal: bool, ffn_chunk: int, R=None, buckets=None, inverse: bool = False,
+                  out1=None, out2=None, ws=None, stream=None, chunk: int = 64):
+    """Reversible layer: forward (x1, x2) -> (y1, y2), or inverse (y1, y2) ->
+    (x1, x2), [B, n, d_model] bf16. weights: w_qk, w_v, w_o [d_model][d_model],
+    w1 [d_ff][d_model], b1 [d_ff], w2 [d_model][d_ff], b2 [d_model] (bf16
+    weights, fp32 biases). Forward without `buckets` hashes them (R needed)
+    and returns them. Returns (out1, out2, buckets)."""
+    W = weights
+    _on_current_device(stream, in1=in1, in2=in2, R=R, buckets=buckets, out1=out1, out2=out2,
+                       ws=ws, **W)
+    B, n, dm = in1.shape
+    dh = dm // heads
+    d_ff = W["w1"].shape[0]
+    for name, t in (("in1", in1), ("in2", in2)):
+        _require(t, name, torch.bfloat16, (B, n, dm))
+    for name, shape in (("w_qk", (dm, dm)), ("w_v", (dm, dm)), ("w_o", (dm, dm)),
+                        ("w1", (d_ff, dm)), ("w2", (dm, d_ff))):
+        _require(W[name], name, torch.bfloat16, shape)
+    for name, shape in (("b1", (d_ff,)), ("b2", (dm,))):
+        if W.get(name) is not None:
+            _require(W[name], name, torch.float32, shape)
+    hash_buckets = not inverse and buckets is None
+    if buckets is None:
+        if inverse:
+            raise ValueError("the inverse needs the forward's bucket ids")
+        if R is None:
+            raise ValueError("either R or buckets is required")
+        buckets = torch.empty((B, heads, rounds, n), dtype=torch.int32, device=in1.device)
+    _require(buckets, "buckets", torch.int32, (B, heads, rounds, n))
+    if R is not None:
+        _require(R, "R", torch.bfloat16, (rounds, dh, n_buckets // 2))
+    desc = LshRevDesc(B, n, dm, heads, dh, d_ff, ffn_chunk, n_buckets, chunk, rounds,
+                      int(bool(causal)), int(hash_buckets))
+    wts = LshRevWeights(*[ctypes.c_void_p(0 if W.get(k) is None else W[k].data_ptr())
+                          for k in ("w_qk", "w_v", "w_o", "w1", "b1", "w2", "b2")])
+    out1 = torch.empty_like(in1) if out1 is None else out1
+    out2 = torch.empty_like(in2) if out2 is None else out2
+    _require(out1, "out1", torch.bfloat16, (B, n, dm))
+    _require(out2, "out2", torch.bfloat16, (B, n, dm))
+    need = ctypes.c_size_t(0)
+    _check(load().lsh_rev_workspace_size(ctypes.byref(desc), ctypes.byref(need)))
+    if ws is None:
+        ws = _scratch(in1.device, stream, need.value)
+    elif ws.numel() < need.value:
+        raise ValueError(f"ws: {need.value} bytes needed, {ws.numel()} given")
+    _check(load().lsh_rev_block(ctypes.byref(desc), int(bool(inverse)), _ptr(in1), _ptr(in2),
+                                ctypes.byref(wts), _ptr(R), _ptr(buckets), _ptr(out1), _ptr(out2),
+                                _ptr(ws), ws.numel(), _stream(stream)))
+    return out1, out2, buckets
 
 
 def _scratch(device, stream, need: int) -> torch.Tensor:

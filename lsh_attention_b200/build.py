@@ -36,7 +36,8 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
         return LIB
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + \
-        ["-o", tmp, os.path.join(CSRC, "lsh_attn.cu"), os.path.join(CSRC, "lsh_attn_noalloc.cu")]
+        ["-o", tmp] + [os.path.join(CSRC, f) for f in ("lsh_attn.cu", "lsh_attn_noalloc.cu",
+                                                        "lsh_rev.cu")]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

@@ -57,6 +57,24 @@ inline bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 tensor in the head-split layout [batch][heads][n][d], seen as 4D
+// (d, n, heads, batch) with tiles of box_inner x box_rows x 1 x 1 and the
+// 128-byte swizzle: a tile of rows (positions) and 64 features of one head.
+inline bool make_tmap_bf16_heads(CUtensorMap* map, const void* base, uint64_t d, uint64_t n,
+                                 uint64_t heads, uint64_t batch, uint32_t box_inner,
+                                 uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {d, n, heads, batch};
+  cuuint64_t strides[3] = {d * 2, d * n * 2, d * n * heads * 2};
+  cuuint32_t box[4] = {box_inner, box_rows, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;

@@ -112,3 +112,25 @@ def make_buckets(w: Workload, seed: int = 7) -> torch.Tensor:
     g = torch.Generator(device="cpu").manual_seed(seed)
     return torch.randint(0, w.n_buckets, (w.batch, w.heads, w.rounds, w.n), generator=g,
                          dtype=torch.int64).to(torch.int32)
+
+
+def make_rev_weights(d_model: int, d_ff: int, seed: int = 2) -> dict:
+    """Weights of a reversible block (bf16, out x in; biases fp32): N(0, 1)
+    scaled by 1/sqrt(fan-in) so activations stay of unit size."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+
+    def w(out_f, in_f):
+        return (torch.randn(out_f, in_f, generator=g) / in_f ** 0.5).to(torch.bfloat16)
+
+    return {"w_qk": w(d_model, d_model), "w_v": w(d_model, d_model), "w_o": w(d_model, d_model),
+            "w1": w(d_ff, d_model), "b1": 0.1 * torch.randn(d_ff, generator=g),
+            "w2": w(d_model, d_ff), "b2": 0.1 * torch.randn(d_model, generator=g)}
+
+
+def make_rev_inputs(batch: int, n: int, d_model: int, seed: int = 3):
+    """The two halves x1, x2 [batch, n, d_model] of a reversible block's input,
+    N(0, 1) in bf16."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    x1 = torch.randn(batch, n, d_model, generator=g).to(torch.bfloat16)
+    x2 = torch.randn(batch, n, d_model, generator=g).to(torch.bfloat16)
+    return x1, x2
