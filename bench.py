@@ -469,6 +469,73 @@ def dense_comparison(dev, K: int = 20, W: int = 3) -> dict:
     return res
 
 
+def time_calls(fn, dev, K: int, W: int) -> float:
+    """Mean ms of fn() over K calls after W, CUDA events on the current stream."""
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(W):
+        fn()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(K):
+        fn()
+    s1.record(stream)
+    torch.cuda.synchronize()
+    return s0.elapsed_time(s1) / K
+
+
+def backward_block(w: I.Workload, dev, K: int = 20, W: int = 3) -> dict:
+    """The backward pass on the main workload (bucket ids from the library's
+    hash, the forward's out and lse, a seeded upstream gradient)."""
+    x_h, v_h = I.make_qkv(w)
+    x, v, R = x_h.to(dev), v_h.to(dev), I.make_rotations(w).to(dev)
+    kw = dict(n_buckets=w.n_buckets, chunk=w.chunk, causal=w.causal)
+    bk = lb.lsh_attn_hash(x, R, w.n_buckets)
+    out, lse = lb.lsh_attn_forward(x, v, None, buckets=bk, **kw)
+    g = torch.Generator(device="cpu").manual_seed(4)
+    dout = torch.randn(x.shape, generator=g).to(x.dtype).to(dev)
+    dx, dv = torch.empty_like(x), torch.empty_like(x)
+    ms = time_calls(lambda: lb.lsh_attn_backward(x, v, bk, out, lse, dout, dx=dx, dv=dv, **kw),
+                    dev, K, W)
+    T = w.batch * w.heads * w.n
+    m = min(w.chunk, w.n)
+    # five products of m queries against 2m keys per chunk and round
+    # (QK^T recomputed, dO V^T, dQ, dK, dV)
+    flops = 5 * 4 * m * w.d * T * w.rounds
+    pk, _ = peaks()
+    return {"config": config_of(w), "ms": round(ms, 4),
+            "tokens_per_s": w.tokens / (ms / 1e3),
+            "TFLOP/s": round(flops / ms / 1e9, 1),
+            "tensor_frac": round(flops / ms / 1e9 / pk["bf16_tflops"], 4),
+            "flops_counted": "5 products of m x 2m x d per chunk and round"}
+
+
+REV_CONFIG = dict(batch=1, n=16384, heads=8, d_head=128, d_ff=4096, rounds=4, n_buckets=256,
+                  ffn_chunk=4096)
+
+
+def reversible_block(dev, K: int = 10, W: int = 3) -> dict:
+    """One reversible layer forward (projections, LSH attention with its own
+    hash, output projection, chunked feed-forward) at d_model 1024."""
+    c = REV_CONFIG
+    dm = c["heads"] * c["d_head"]
+    Wt = {k: v.to(dev) for k, v in I.make_rev_weights(dm, c["d_ff"]).items()}
+    x1, x2 = (t.to(dev) for t in I.make_rev_inputs(c["batch"], c["n"], dm))
+    wl = I.Workload("rev", c["batch"], c["heads"], c["n"], c["d_head"], c["n_buckets"], 64,
+                    c["rounds"], True, "bf16")
+    R = I.make_rotations(wl).to(dev)
+    kw = dict(heads=c["heads"], n_buckets=c["n_buckets"], rounds=c["rounds"], causal=True,
+              ffn_chunk=c["ffn_chunk"])
+    y1, y2 = torch.empty_like(x1), torch.empty_like(x2)
+    ms = time_calls(lambda: lb.lsh_rev_block(x1, x2, Wt, R=R, out1=y1, out2=y2, **kw), dev, K, W)
+    rows = c["batch"] * c["n"]
+    gemm_flops = 2 * rows * dm * dm * 3 + 2 * 2 * rows * dm * c["d_ff"]
+    return {"config": dict(c, d_model=dm, chunk=64, causal=True), "ms": round(ms, 4),
+            "tokens_per_s": rows / (ms / 1e3),
+            "gemm_GFLOP": round(gemm_flops / 1e9, 1),
+            "gemm_TFLOP/s_if_all_time": round(gemm_flops / ms / 1e9, 1)}
+
+
 def run_ours(args, w):
     world, rank, local = dist_setup("nccl")
     torch.cuda.set_device(local)
@@ -494,6 +561,8 @@ def run_ours(args, w):
                            "kernels_ms": {kn: round(t, 4) for kn, t in mx["kernel_ms"].items()}}
             del mx
         extra["dense_baseline"] = dense_comparison(dev)
+        extra["backward"] = backward_block(w, dev)
+        extra["reversible_layer"] = reversible_block(dev)
     if rank != 0:
         return
     stages, roof = roofline_block(w, m["kernel_ms"], total_ms / 1e3)

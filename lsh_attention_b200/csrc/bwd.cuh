@@ -119,26 +119,33 @@ struct BwdArgs {
   float* dv;               // k_bwd_dkv: [S][n][d] dv, slot order
   WsHeader* hdr;
   int n, rounds, pairs_per_seg;
+  int oob;                 // a row index past x, v and g (BH * n): reads as zero
   int64_t units;           // BH * pairs_per_seg * rounds
 };
 
 constexpr int kNoPos = 0x7fffffff;
 
-// Copies `rows` rows of src (position order, row `pos(r)`) into a swizzled
-// K-major tile [KH][rows][128 B] by cp.async, all threads of the CTA; a row
-// whose position is kNoPos is zero-filled.
+// Warp 0 gathers `rows` rows of a [BH * n][D] tensor (row rbase + pos(r), or
+// a row past the tensor, which reads as zero, for kNoPos) into a swizzled
+// K-major tile [KH][rows][128 B] with TMA (tile::gather4: four rows per
+// instruction, each landing by its shared-memory address); completion is
+// counted on `bar`, whose expected bytes the caller sets.
 template <int D, typename PosFn>
-__device__ __forceinline__ void bwd_load_rows(unsigned char* tile, int rows,
-                                              const __nv_bfloat16* src, PosFn pos) {
-  constexpr int CPR = D / 8;  // 16-byte pieces per row
-  const uint32_t box = (uint32_t)rows * 128;
-  for (int e = threadIdx.x; e < rows * CPR; e += blockDim.x) {
-    const int row = e / CPR, piece = e % CPR;
-    const int kh = piece >> 3, cc = piece & 7;
-    const int p = pos(row);
-    const bool valid = p != kNoPos;
-    const __nv_bfloat16* s = valid ? src + (int64_t)p * D + piece * 8 : src;
-    sm100::cp_async16_zfill(tile + kh * box + row * 128 + ((cc ^ (row & 7)) << 4), s, valid);
+__device__ __forceinline__ void bwd_gather(unsigned char* tile, int rows, const CUtensorMap* map,
+                                           uint64_t* bar, int rbase, int oob, PosFn pos) {
+  constexpr int KH = D / 64;
+  const int lane = threadIdx.x & 31;
+  for (int g = lane; g < rows / 4; g += 32) {
+    int r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int p = pos(4 * g + j);
+      r[j] = p == kNoPos ? oob : rbase + p;
+    }
+#pragma unroll
+    for (int kh = 0; kh < KH; ++kh)
+      sm100::tma_gather4_2d(tile + kh * rows * 128 + 4 * g * 128, map, bar, kh * 64, r[0], r[1],
+                            r[2], r[3]);
   }
 }
 
@@ -164,7 +171,9 @@ inline size_t bwd_dq_smem() {
 // Query-stationary: dQ of the 128 queries of a chunk pair.
 // TMEM: S [0, 192) (dS' bf16 over [0, 96)), dPraw [192, 384), dQ [384, 384 + d).
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(kBwdWarps * 32, 1) k_bwd_dq(BwdArgs a) {
+__global__ void __launch_bounds__(kBwdWarps * 32, 1)
+    k_bwd_dq(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmv,
+             const __grid_constant__ CUtensorMap tmg, BwdArgs a) {
   using namespace sm100;
   constexpr int KH = D / 64;
   constexpr uint32_t XBOX = 192 * 128, GBOX = 128 * 128;
@@ -181,11 +190,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) k_bwd_dq(BwdArgs a) {
   uint64_t* bar_q = bars + 1;   // dQ MMA done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* bad = reinterpret_cast<volatile int*>(bars + 3);
+  uint64_t* bar_ld = bars + 4;  // the unit's rows landed (tx)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     mbar_init(bar_sp, 1);
     mbar_init(bar_q, 1);
+    mbar_init(bar_ld, 1);
     *bad = 0;
     fence_mbar_init();
   }
@@ -219,12 +230,16 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) k_bwd_dq(BwdArgs a) {
       }
     }
     __syncthreads();
-    const __nv_bfloat16* xb = a.x + bh * a.n * D;
-    bwd_load_rows<D>(xt, 192, xb, [&](int r) { return __float_as_int(kt[r].w); });
-    bwd_load_rows<D>(vt, 192, a.v + bh * a.n * D, [&](int r) { return __float_as_int(kt[r].w); });
-    bwd_load_rows<D>(gt, 128, a.g + bh * a.n * D, [&](int r) { return __float_as_int(qt[r].x); });
-    cp_async_wait_all();
-    fence_proxy_async_smem();
+    if (warp == 0) {
+      if (lane == 0) mbar_expect_tx(bar_ld, (uint32_t)(KH * (2 * XBOX + GBOX)));
+      __syncwarp();
+      const int rb = (int)(bh * a.n);
+      auto kpos = [&](int r) { return __float_as_int(kt[r].w); };
+      bwd_gather<D>(xt, 192, &tmx, bar_ld, rb, a.oob, kpos);
+      bwd_gather<D>(vt, 192, &tmv, bar_ld, rb, a.oob, kpos);
+      bwd_gather<D>(gt, 128, &tmg, bar_ld, rb, a.oob, [&](int r) { return __float_as_int(qt[r].x); });
+    }
+    if (!mbar_wait(bar_ld, it & 1)) *bad = 1;
     tc_fence_before();
     __syncthreads();
     // ---- S = Q K^T, dPraw = G_q V^T
@@ -341,7 +356,9 @@ inline size_t bwd_dkv_smem() {
 // TMEM: S^T [0, 128) (P w bf16 over [0, 64)), dPraw^T [128, 256) (dS' bf16
 // over [128, 192)), dV [256, 256 + d), G [384, 384 + d).
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(kBwdWarps * 32, 1) k_bwd_dkv(BwdArgs a) {
+__global__ void __launch_bounds__(kBwdWarps * 32, 1)
+    k_bwd_dkv(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmv,
+              const __grid_constant__ CUtensorMap tmg, BwdArgs a) {
   using namespace sm100;
   constexpr int KH = D / 64;
   constexpr uint32_t XBOX = 192 * 128, VBOX = 128 * 128;
@@ -358,11 +375,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) k_bwd_dkv(BwdArgs a) {
   uint64_t* bar_acc = bars + 1;  // dV and G MMAs of a pass done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
   volatile int* bad = reinterpret_cast<volatile int*>(bars + 3);
+  uint64_t* bar_ld = bars + 4;  // the unit's rows landed (tx)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     mbar_init(bar_sp, 1);
     mbar_init(bar_acc, 1);
+    mbar_init(bar_ld, 1);
     *bad = 0;
     fence_mbar_init();
   }
@@ -373,8 +392,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) k_bwd_dkv(BwdArgs a) {
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_dp = tmem + 128, tm_dv = tmem + 256, tm_g = tmem + 384;
 
-  int phase = 0;  // completions of each barrier so far (both complete twice per unit)
-  for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x) {
+  int phase = 0;  // completions of bar_sp and bar_acc so far (twice per unit)
+  int it = 0;     // units so far (bar_ld completes once per unit)
+  for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x, ++it) {
     int64_t bh, seg;
     int c0;
     bwd_unit(a, u, bh, seg, c0);
@@ -391,12 +411,16 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1) k_bwd_dkv(BwdArgs a) {
       }
     }
     __syncthreads();
-    const int64_t ho = bh * a.n * D;
-    bwd_load_rows<D>(xt, 192, a.x + ho, [&](int r) { return __float_as_int(qt[r].x); });
-    bwd_load_rows<D>(vt, 128, a.v + ho, [&](int r) { return __float_as_int(kt[r].w); });
-    bwd_load_rows<D>(gt, 192, a.g + ho, [&](int r) { return __float_as_int(qt[r].x); });
-    cp_async_wait_all();
-    fence_proxy_async_smem();
+    if (warp == 0) {
+      if (lane == 0) mbar_expect_tx(bar_ld, (uint32_t)(KH * (2 * XBOX + VBOX)));
+      __syncwarp();
+      const int rb = (int)(bh * a.n);
+      auto qpos = [&](int r) { return __float_as_int(qt[r].x); };
+      bwd_gather<D>(xt, 192, &tmx, bar_ld, rb, a.oob, qpos);
+      bwd_gather<D>(vt, 128, &tmv, bar_ld, rb, a.oob, [&](int r) { return __float_as_int(kt[r].w); });
+      bwd_gather<D>(gt, 192, &tmg, bar_ld, rb, a.oob, qpos);
+    }
+    if (!mbar_wait(bar_ld, it & 1)) *bad = 1;
     tc_fence_before();
     __syncthreads();
     for (int pass = 0; pass < 2; ++pass, ++phase) {

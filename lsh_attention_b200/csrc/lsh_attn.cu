@@ -570,16 +570,23 @@ lsh_status check_bwd(const lsh_attn_desc* desc, Dims* D, BwdLayout* L) {
 }
 
 template <int DD, bool CAUSAL>
-lsh_status launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
+lsh_status launch_bwd_tc(const BwdArgs& a, const Dims& D, cudaStream_t st) {
   const int sms = sm_count();
   const unsigned grid = (unsigned)std::min<int64_t>(a.units, sms);
+  // x, v and g in position order, one-row boxes for the gathers
+  CUtensorMap tmx, tmv, tmg;
+  const uint64_t prow = (uint64_t)D.BH * D.n;
+  if (!make_tmap_bf16_2d(&tmx, a.x, DD, prow, (uint64_t)DD * 2, 64, 1) ||
+      !make_tmap_bf16_2d(&tmv, a.v, DD, prow, (uint64_t)DD * 2, 64, 1) ||
+      !make_tmap_bf16_2d(&tmg, a.g, DD, prow, (uint64_t)DD * 2, 64, 1))
+    return LSH_ERR_CUDA;
   {
     auto kern = k_bwd_dq<DD, CAUSAL>;
     const size_t smem = bwd_dq_smem<DD>();
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return LSH_ERR_CUDA;
-    kern<<<grid, kBwdWarps * 32, smem, st>>>(a);
+    kern<<<grid, kBwdWarps * 32, smem, st>>>(tmx, tmv, tmg, a);
   }
   {
     auto kern = k_bwd_dkv<DD, CAUSAL>;
@@ -587,7 +594,7 @@ lsh_status launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return LSH_ERR_CUDA;
-    kern<<<grid, kBwdWarps * 32, smem, st>>>(a);
+    kern<<<grid, kBwdWarps * 32, smem, st>>>(tmx, tmv, tmg, a);
   }
   return last_cuda();
 }
@@ -632,7 +639,9 @@ lsh_status backward_d(const Dims& D, const BwdLayout& L, const void* x, const vo
   a.rounds = D.rounds;
   a.pairs_per_seg = (D.n / kAttnM + 1) / 2;
   a.units = D.S * a.pairs_per_seg;
-  if ((s = D.causal ? launch_bwd_tc<DD, true>(a, st) : launch_bwd_tc<DD, false>(a, st)) != LSH_OK)
+  a.oob = (int)(D.BH * D.n);
+  if ((s = D.causal ? launch_bwd_tc<DD, true>(a, D, st) : launch_bwd_tc<DD, false>(a, D, st)) !=
+      LSH_OK)
     return s;
   k_bwd_unsort<T, DD><<<(unsigned)std::min<int64_t>((pos_total + 7) / 8, 8 * sms), 256, 0, st>>>(
       inv, a.dq, a.dxk, a.dv, static_cast<T*>(dx), static_cast<T*>(dv), D.n, D.rounds, pos_total);
