@@ -279,6 +279,35 @@ lsh_status lsh_rev_block(const lsh_rev_desc *desc, int inverse, const void *in1,
                          void *out1, void *out2, void *workspace, size_t workspace_bytes,
                          void *stream);
 
+/* The in-bucket top-k variant of LSH attention ("Reformer re-reading",
+ * §2.2), a second workload beside lsh_attn_forward: per round l, bucket(x) =
+ * (sum_t [proj_l[:, t] . x > 0] 2^t) mod n_buckets over n_bits projections;
+ * every query ranks the keys of its bucket (causal: positions <= its own) by
+ * the chunked attention's logit x_i . x_j / (||x_j|| sqrt(d)) (-1e5 for
+ * itself; higher first, lower position on ties) and keeps the top_k; the
+ * candidates are the union over rounds, attended with one softmax of those
+ * logits. Bucket bits and top-k sets are decided in fp64 (sums in increasing
+ * feature order, no fused multiply-add); the softmax runs in fp32. */
+typedef struct {
+    int32_t batch, heads, n, d;  /* d in {64, 128} */
+    int32_t n_buckets;           /* K: even, 2 .. 4096 */
+    int32_t n_bits;              /* m projections per round, 1 .. 32 */
+    int32_t top_k;               /* 1 .. 32 */
+    int32_t rounds;              /* L: 1 .. 8 */
+    int32_t causal;
+} lsh_topk_desc;
+
+/* Workspace bytes lsh_topk_forward needs for `desc`. */
+lsh_status lsh_topk_workspace_size(const lsh_topk_desc *desc, size_t *bytes);
+
+/* x, v, out [B][H][n][d] bf16; proj [rounds][d][n_bits] bf16; lse [B][H][n]
+ * fp32; cand (optional, else kept in the workspace) [B][H][rounds][n][top_k]
+ * int32: each round's top-k positions, best first, -1 past the kept ones.
+ * Conventions as for lsh_attn_forward. */
+lsh_status lsh_topk_forward(const lsh_topk_desc *desc, const void *x, const void *v,
+                            const void *proj, void *out, float *lse, int32_t *cand,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
 /* Static, human-readable name of a status code. */
 const char *lsh_attn_status_string(lsh_status status);
 

@@ -28,7 +28,8 @@ EXPORTS = ("lsh_attn_workspace_size", "lsh_attn_hash", "lsh_attn_sort", "lsh_att
            "lsh_attn_sort_noalloc", "lsh_attn_selftest_wait_timeout",
            "lsh_attn_dense_workspace_size", "lsh_attn_dense_forward",
            "lsh_attn_backward_workspace_size", "lsh_attn_backward", "lsh_rev_workspace_size",
-           "lsh_rev_block", "lsh_attn_status_string")
+           "lsh_rev_block", "lsh_topk_workspace_size", "lsh_topk_forward",
+           "lsh_attn_status_string")
 
 
 class LshAttnDesc(ctypes.Structure):
@@ -49,6 +50,11 @@ class LshRevDesc(ctypes.Structure):
 
 class LshRevWeights(ctypes.Structure):
     _fields_ = [(k, ctypes.c_void_p) for k in ("w_qk", "w_v", "w_o", "w1", "b1", "w2", "b2")]
+
+
+class LshTopkDesc(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_int32) for k in
+                ("batch", "heads", "n", "d", "n_buckets", "n_bits", "top_k", "rounds", "causal")]
 
 
 class LshAttnError(RuntimeError):
@@ -95,6 +101,10 @@ def load() -> ctypes.CDLL:
             lib.lsh_rev_block.argtypes = [ctypes.POINTER(LshRevDesc), ctypes.c_int, vp, vp,
                                           ctypes.POINTER(LshRevWeights), vp, vp, vp, vp, vp, sz,
                                           vp]
+            lib.lsh_topk_workspace_size.argtypes = [ctypes.POINTER(LshTopkDesc),
+                                                    ctypes.POINTER(sz)]
+            lib.lsh_topk_forward.argtypes = [ctypes.POINTER(LshTopkDesc), vp, vp, vp, vp, vp, vp,
+                                             vp, sz, vp]
             lib.lsh_attn_status_string.argtypes = [ctypes.c_int]
             lib.lsh_attn_status_string.restype = ctypes.c_char_p
             for f in EXPORTS[:-1]:
@@ -368,6 +378,35 @@ def lsh_rev_block(in1, in2, weights: dict, *, heads: int, n_buckets: int, rounds
                                 ctypes.byref(wts), _ptr(R), _ptr(buckets), _ptr(out1), _ptr(out2),
                                 _ptr(ws), ws.numel(), _stream(stream)))
     return out1, out2, buckets
+
+
+def lsh_topk_forward(x, v, proj, *, n_buckets: int, top_k: int, causal: bool,
+                     return_candidates: bool = False, out=None, lse=None, ws=None, stream=None):
+    """The in-bucket top-k variant: x, v [B, H, n, d] bf16, proj [rounds, d,
+    n_bits] bf16. Returns (out, lse [B, H, n]) and, if asked, the candidates
+    [B, H, rounds, n, top_k] int32 (-1 past the kept ones)."""
+    _on_current_device(stream, x=x, v=v, proj=proj, out=out, lse=lse, ws=ws)
+    B, H, n, d = x.shape
+    L, _, m = proj.shape
+    _require(x, "x", torch.bfloat16, None)
+    _require(v, "v", torch.bfloat16, tuple(x.shape))
+    _require(proj, "proj", torch.bfloat16, (L, d, m))
+    desc = LshTopkDesc(B, H, n, d, n_buckets, m, top_k, L, int(bool(causal)))
+    out = torch.empty_like(x) if out is None else out
+    lse = torch.empty((B, H, n), dtype=torch.float32, device=x.device) if lse is None else lse
+    _require(out, "out", torch.bfloat16, tuple(x.shape))
+    _require(lse, "lse", torch.float32, (B, H, n))
+    cand = (torch.empty((B, H, L, n, top_k), dtype=torch.int32, device=x.device)
+            if return_candidates else None)
+    need = ctypes.c_size_t(0)
+    _check(load().lsh_topk_workspace_size(ctypes.byref(desc), ctypes.byref(need)))
+    if ws is None:
+        ws = _scratch(x.device, stream, need.value)
+    elif ws.numel() < need.value:
+        raise ValueError(f"ws: {need.value} bytes needed, {ws.numel()} given")
+    _check(load().lsh_topk_forward(ctypes.byref(desc), _ptr(x), _ptr(v), _ptr(proj), _ptr(out),
+                                   _ptr(lse), _ptr(cand), _ptr(ws), ws.numel(), _stream(stream)))
+    return (out, lse, cand) if return_candidates else (out, lse)
 
 
 def _scratch(device, stream, need: int) -> torch.Tensor:

@@ -19,6 +19,7 @@
 #include "merge.cuh"
 #include "sort.cuh"
 #include "tma_host.cuh"
+#include "topk.cuh"
 
 namespace {
 
@@ -648,6 +649,66 @@ lsh_status backward_d(const Dims& D, const BwdLayout& L, const void* x, const vo
   return last_cuda();
 }
 
+// ---------------------------------------------------------------- top-k variant
+struct TopkLayout {
+  size_t header, bucket, perm, inv, hist, cand, total;
+};
+
+lsh_status check_topk(const lsh_topk_desc* t, Dims* D, TopkLayout* L) {
+  if (!t) return LSH_ERR_INVALID_ARG;
+  const lsh_topk_desc& q = *t;
+  if (q.batch < 1 || q.heads < 1 || q.n < 1 || q.d < 1 || q.n_buckets < 1 || q.n_bits < 1 ||
+      q.top_k < 1 || q.rounds < 1 || (q.causal != 0 && q.causal != 1))
+    return LSH_ERR_INVALID_ARG;
+  if ((q.d != 64 && q.d != 128) || q.n_bits > kTopkMaxBits || q.top_k > kTopkMaxK ||
+      q.rounds > kTopkMaxRounds)
+    return LSH_ERR_UNSUPPORTED;
+  // the counting sort takes an even bucket count in [2, 4096]
+  const lsh_attn_desc ad{q.batch, q.heads, q.n, q.d, q.n_buckets, 1, q.rounds, q.causal, LSH_BF16};
+  lsh_status s = check_desc(&ad, D, false);
+  if (s != LSH_OK) return s;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const size_t sn = (size_t)D->S * D->n;
+  L->header = take(sizeof(WsHeader));
+  L->bucket = take(sn * 4);
+  L->perm = take(sn * 4);
+  L->inv = take(sn * 4);
+  L->hist = take((size_t)D->S * D->nb * D->tiles * 4);
+  L->cand = take(sn * q.top_k * 4);
+  L->total = off;
+  return LSH_OK;
+}
+
+template <int DD>
+lsh_status topk_forward_d(const Dims& D, const TopkLayout& L, const lsh_topk_desc& q,
+                          const void* x, const void* v, const void* proj, void* out, float* lse,
+                          int32_t* cand, void* ws, cudaStream_t st) {
+  using T = __nv_bfloat16;
+  const int sms = sm_count();
+  int32_t* bucket = at<int32_t>(ws, L.bucket);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  const int64_t hash_total = D.S * D.n;
+  k_tk_hash<DD><<<(unsigned)std::min<int64_t>((hash_total + 255) / 256, 16 * sms), 256, 0, st>>>(
+      static_cast<const T*>(x), static_cast<const T*>(proj), bucket, D.n, D.rounds, q.n_bits,
+      q.n_buckets, hash_total);
+  lsh_status s = launch_sort<T>(D, bucket, x, v, perm, at<int32_t>(ws, L.inv), nullptr, nullptr,
+                                nullptr, at<int32_t>(ws, L.hist), at<WsHeader>(ws, L.header), st);
+  if (s != LSH_OK) return s;
+  const int64_t sel_total = D.S * D.n;  // warps
+  k_tk_select<DD><<<(unsigned)std::min<int64_t>((sel_total + 7) / 8, 16 * sms), 256, 0, st>>>(
+      static_cast<const T*>(x), bucket, perm, cand, D.n, D.rounds, q.top_k, q.causal, sel_total);
+  const int64_t att_total = D.BH * D.n;
+  k_tk_attend<DD><<<(unsigned)std::min<int64_t>((att_total + 7) / 8, 16 * sms), 256, 0, st>>>(
+      static_cast<const T*>(x), static_cast<const T*>(v), cand, static_cast<T*>(out), lse, D.n,
+      D.rounds, q.top_k, att_total);
+  return last_cuda();
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ C ABI
@@ -795,6 +856,32 @@ lsh_status lsh_attn_backward(const lsh_attn_desc* desc, const void* x, const voi
   if ((s = reset_header(ws, st)) != LSH_OK) return s;
   return D.d == 64 ? backward_d<64>(D, L, x, v, buckets, out, lse, dout, dlse, dx, dv, ws, st)
                    : backward_d<128>(D, L, x, v, buckets, out, lse, dout, dlse, dx, dv, ws, st);
+}
+
+lsh_status lsh_topk_workspace_size(const lsh_topk_desc* desc, size_t* bytes) {
+  Dims D;
+  TopkLayout L;
+  lsh_status s = check_topk(desc, &D, &L);
+  if (s != LSH_OK) return s;
+  if (!bytes) return LSH_ERR_INVALID_ARG;
+  *bytes = L.total;
+  return LSH_OK;
+}
+
+lsh_status lsh_topk_forward(const lsh_topk_desc* desc, const void* x, const void* v,
+                            const void* proj, void* out, float* lse, int32_t* cand, void* ws,
+                            size_t ws_bytes, void* stream) {
+  Dims D;
+  TopkLayout L;
+  lsh_status s = check_topk(desc, &D, &L);
+  if (s != LSH_OK) return s;
+  if (!x || !v || !proj || !out || !lse) return LSH_ERR_INVALID_ARG;
+  if (!ws || ((uintptr_t)ws & 255) != 0 || ws_bytes < L.total) return LSH_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = reset_header(ws, st)) != LSH_OK) return s;
+  int32_t* c = cand ? cand : at<int32_t>(ws, L.cand);
+  return D.d == 64 ? topk_forward_d<64>(D, L, *desc, x, v, proj, out, lse, c, ws, st)
+                   : topk_forward_d<128>(D, L, *desc, x, v, proj, out, lse, c, ws, st);
 }
 
 lsh_status lsh_attn_get_diag(const void* ws, void* stream, lsh_attn_diag* diag) {

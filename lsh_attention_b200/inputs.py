@@ -134,3 +134,10 @@ def make_rev_inputs(batch: int, n: int, d_model: int, seed: int = 3):
     x1 = torch.randn(batch, n, d_model, generator=g).to(torch.bfloat16)
     x2 = torch.randn(batch, n, d_model, generator=g).to(torch.bfloat16)
     return x1, x2
+
+
+def make_topk_projections(rounds: int, d: int, n_bits: int, seed: int = 1) -> torch.Tensor:
+    """SimHash projections of the top-k variant, [rounds, d, n_bits], N(0, 1)
+    rounded to bf16."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return torch.randn(rounds, d, n_bits, generator=g).to(torch.bfloat16)
