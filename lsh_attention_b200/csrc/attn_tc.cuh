@@ -25,6 +25,13 @@
 //               128 bytes per instruction, landing in the 128-byte-swizzled
 //               K-major tile by their shared-memory address); a slot outside
 //               [0, n) reads as zero.
+//   warps 10-11 v loaders: the 192 v rows, at the positions of the ring, by
+//               16-byte cp.async copies into the swizzled tile of the P.V
+//               product; when a thread's copies have landed it fences them for
+//               the async proxy (the tensor cores read shared memory through
+//               it) and arrives. Gathering x by TMA and v by cp.async at once
+//               uses both copy paths, each of which alone issues too slowly to
+//               keep up with the tensor cores.
 //   warp 1      tcgen05.mma: S(u+1) = Q K^T into TMEM S[s], then O(u) = P V
 //               with P read from TMEM, so S of the next unit is ready when
 //               the softmax warps finish the current one. The x tile is free
@@ -53,7 +60,7 @@ namespace lsh {
 
 constexpr int kAttnM = 64;      // chunk length served by this kernel
 constexpr int kAttnKeys = 192;  // key window of a pair of chunks
-constexpr int kAttnWarps = 10;
+constexpr int kAttnWarps = 12;
 constexpr int kAttnStats = 4;   // row-sum slots between softmax and epilogue
 constexpr int kAttnRing = 4;    // metadata ring depth
 // Above this bound (log2 units) the stabiliser could push exp2 below the
@@ -86,8 +93,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnWarps * 32, 1)
-    k_attn_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmv,
-              const __grid_constant__ CUtensorMap tmo, AttnTcArgs a) {
+    k_attn_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmo,
+              AttnTcArgs a) {
   using namespace sm100;
   constexpr int KH = D / 64;
   constexpr uint32_t BOX = kAttnKeys * 128;
@@ -106,7 +113,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(rstat + kAttnStats * 128);
   uint64_t* xfull = bars + 0;    // [2] x rows landed (tx)
   uint64_t* xfree = bars + 2;    // [2] S MMA done with the x tile
-  uint64_t* vfull = bars + 4;    // [2] v rows landed (tx)
+  uint64_t* vfull = bars + 4;    // [2] v rows landed (64 v-loader threads)
   uint64_t* vfree = bars + 6;    // [2] PV MMA done with the v tile
   uint64_t* sfull = bars + 8;    // [2] S MMA done
   uint64_t* pready = bars + 10;  // [2] P written (4 softmax warps)
@@ -115,7 +122,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   uint64_t* ofree = bars + 15;   // 4 epilogue warps done reading O
   uint64_t* statf = bars + 16;   // [4] row sums written (4 softmax warps)
   uint64_t* mfull = bars + 20;   // [ring] metadata written (32 producer lanes)
-  uint64_t* mfree = bars + 24;   // [ring] 4 softmax warps done with it
+  uint64_t* mfree = bars + 24;   // [ring] 4 softmax warps and 2 v-loader warps done with it
   uint64_t* drain = bars + 28;   // MMA issuer: every issued MMA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 29);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 30);
@@ -129,7 +136,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(xfull + i, 1);
       mbar_init(xfree + i, 1);
-      mbar_init(vfull + i, 1);
+      mbar_init(vfull + i, 64);
       mbar_init(vfree + i, 1);
       mbar_init(sfull + i, 1);
       mbar_init(pready + i, 4);
@@ -140,7 +147,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     for (int i = 0; i < kAttnStats; ++i) mbar_init(statf + i, 4);
     for (int i = 0; i < kAttnRing; ++i) {
       mbar_init(mfull + i, 32);
-      mbar_init(mfree + i, 4);
+      mbar_init(mfree + i, 4 + 2);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -174,7 +181,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&tmx);
-      prefetch_tensormap(&tmv);
     }
     const int oob = (int)(a.units / a.rounds / a.pairs_per_seg) * a.n;  // rows: a row past them
     // positions (perm) of a unit's window rows lane + 32 t, and their logit
@@ -206,7 +212,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     scale_of(0, p0, s0);
     scale_of(1, p1, s1);
     perm_of(2, p2);
-    int lastx[2] = {-1, -1}, lastv[2] = {-1, -1};
+    int lastx[2] = {-1, -1};
     bool ok = true;
     for (int i = 0; i < nu; ++i) {
       const int s = i & 1, k = i >> 1, m = i & (kAttnRing - 1), km = i / kAttnRing;
@@ -254,25 +260,13 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       }
       scale_of(i + 2, p1, s1);  // p1 now holds unit i + 2's positions
       perm_of(i + 3, p2);
-      // v tile s free (PV of unit i - 2 done)
-      got = k == 0 || mbar_wait(vfree + s, (k - 1) & 1);
-      if (__any_sync(0xffffffffu, !got || *abort_flag)) {
-        ok = __all_sync(0xffffffffu, got);
-        break;
-      }
-      if (lane == 0) mbar_expect_tx(vfull + s, TILE);
-      __syncwarp();
-      gather(&tmv, vt + s * TILE, vfull + s);
-      if (lane == 0) lastv[s] = k;
     }
     if (lane == 0) {
       if (!ok) fail();
       // No copy may still be writing this CTA's shared memory when it exits:
       // wait (bounded) for the last phase issued on every stage.
       for (int s = 0; s < 2; ++s)
-        if ((lastx[s] >= 0 && !mbar_wait(xfull + s, lastx[s] & 1)) ||
-            (lastv[s] >= 0 && !mbar_wait(vfull + s, lastv[s] & 1)))
-          *drain_fail = 1;
+        if (lastx[s] >= 0 && !mbar_wait(xfull + s, lastx[s] & 1)) *drain_fail = 1;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -420,7 +414,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         mbar_arrive(mfree + m);
       }
     }
-  } else {
+  } else if (warp < 10) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -484,6 +478,42 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       }
     }
     if (lane == 0) bulk_wait_all();
+  } else {
+    // ------------------------------------------------------------ v loaders
+    constexpr int CPR = KH * 8;      // 16-byte pieces per row
+    constexpr int RSTEP = 64 / CPR;  // rows between a thread's pieces
+    const int lt = tid - 10 * 32;    // 0..63
+    const int piece = lt % CPR, kh = piece >> 3, cc = piece & 7;
+    for (int i = 0; i < nu; ++i) {
+      const int s = i & 1, k = i >> 1, m = i & (kAttnRing - 1), km = i / kAttnRing;
+      // ring slot m written for unit i, v tile s free (PV of unit i - 2 done)
+      const bool got =
+          mbar_wait(mfull + m, km & 1) && (k == 0 || mbar_wait(vfree + s, (k - 1) & 1));
+      if (!got) fail();
+      // both loader warps stop together (a failure anywhere sets abort_flag)
+      if (bar_sync_any(3, 64, !got || *abort_flag)) break;
+      int64_t bh, seg;
+      int c0;
+      unit_of(i, bh, seg, c0);
+      const float2* kt = ktab + m * kAttnKeys;
+      const unsigned char* v0 = reinterpret_cast<const unsigned char*>(a.v);
+      const unsigned char* rows = v0 + (bh * a.n) * (int64_t)(D * 2) + piece * 16;
+      unsigned char* dst = vt + s * TILE + kh * BOX;
+#pragma unroll 4
+      for (int row = lt / CPR; row < kAttnKeys; row += RSTEP) {
+        const int pos = __float_as_int(kt[row].y);
+        const bool valid = pos != kNoKey;
+        cp_async16_zfill(dst + row * 128 + ((cc ^ (row & 7)) << 4),
+                         valid ? rows + (int64_t)pos * (D * 2) : v0, valid);
+      }
+      cp_async_commit();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(mfree + m);  // done reading the ring slot
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      mbar_arrive(vfull + s);
+    }
+    cp_async_wait_all();  // no copy of this thread still writes shared memory at exit
   }
   tc_fence_before();
   __syncthreads();

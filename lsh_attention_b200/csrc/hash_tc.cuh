@@ -292,9 +292,13 @@ struct BatchLead {
     const bool lead = bm > m1;        // the earlier batch keeps the lead on a tie
     m2o = fmaxf(m2o, fminf(bm, m1));  // the batch that does not lead
     m1 = fmaxf(m1, bm);
-    j0 = lead ? jb : j0;
+    // the copy is branched over rather than selected element by element:
+    // measured cheaper even when every lane leads
+    if (lead) {
+      j0 = jb;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) s[k] = lead ? w[k] : s[k];
+      for (int k = 0; k < 16; ++k) s[k] = w[k];
+    }
   }
   // Largest |p|, second largest, argmax column and its signed value; all
   // zero when no batch was added.
