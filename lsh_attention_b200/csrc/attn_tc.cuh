@@ -11,39 +11,39 @@
 // Work unit: a pair of chunks (c0, c0+1) of one (batch, head, round). Its 128
 // queries are slots [64 c0, 64 c0 + 128) and its key window is slots
 // [64 (c0-1), 64 (c0+2)): the queries are rows 64..191 of the key tile.
-// Units are numbered (batch, head) first, then chunk pair, then round, and
-// CTA c of G takes units c, c + G, c + 2G, ...: at any time the CTAs work on
-// neighbouring units of one (batch, head), so every round reads that head's
-// rows while they sit in L2 and HBM delivers each row about once.
+// Units of a (batch, head) are numbered round first, then chunk pair; the
+// CTAs split every (batch, head)'s units into contiguous runs and walk the
+// (batch, head)s in order. So at any time the CTAs work on one (batch,
+// head), whose rows all rounds read while they sit in L2 (HBM delivers each
+// row about once), and consecutive units of a CTA are consecutive chunk
+// pairs of one round: the first 64 rows of a window are the last 64 of the
+// previous window, copied inside shared memory instead of gathered again
+// (row r + 128 has the swizzle phase of row r), a third fewer rows to fetch.
 //
-// One persistent CTA per SM, 10 warps:
-//   warp 0      producer: the window's positions (perm) and key norms
+// One persistent CTA per SM, 13 warps:
+//   warps 0-1   x loaders: the window's positions (perm) and key norms
 //               (1/||x|| by position) are loaded into registers two and one
-//               units ahead, written to a 4-deep ring of (logit scale,
-//               position) per key, and the 192 x rows and then the 192 v rows
-//               are gathered by position with TMA (tile::gather4: four rows of
-//               128 bytes per instruction, landing in the 128-byte-swizzled
-//               K-major tile by their shared-memory address); a slot outside
-//               [0, n) reads as zero.
-//   warps 10-11 v loaders: the 192 v rows, at the positions of the ring, by
-//               16-byte cp.async copies into the swizzled tile of the P.V
-//               product; when a thread's copies have landed it fences them for
-//               the async proxy (the tensor cores read shared memory through
-//               it) and arrives. Gathering x by TMA and v by cp.async at once
-//               uses both copy paths, each of which alone issues too slowly to
-//               keep up with the tensor cores.
-//   warp 1      tcgen05.mma: S(u+1) = Q K^T into TMEM S[s], then O(u) = P V
+//               units ahead and written to a 4-deep ring of (logit scale,
+//               position) per key; the x rows not carried over go by 16-byte
+//               cp.async copies to their places in the 128-byte-swizzled
+//               K-major tile (a slot outside [0, n) reads as zero). When a
+//               thread's copies have landed it fences them for the async
+//               proxy (the tensor cores read shared memory through it) and
+//               arrives.
+//   warps 2-3   v loaders: the same for the v rows, at the positions of the
+//               ring, into the tile of the P.V product.
+//   warp 4      tcgen05.mma: S(u+1) = Q K^T into TMEM S[s], then O(u) = P V
 //               with P read from TMEM, so S of the next unit is ready when
 //               the softmax warps finish the current one. The x tile is free
 //               again as soon as S is computed (the ring keeps the metadata).
-//   warps 2-5   softmax, one query row per thread, one pass: logits in log2
+//   warps 5-8   softmax, one query row per thread, one pass: logits in log2
 //               units are bounded by ||q|| log2(e) / sqrt(d) (keys have unit
 //               length), which serves as the stabiliser, so every probability
 //               is exp2(l - bound) <= 1 and is written to TMEM (bf16, over the
 //               dead S columns) as soon as it is computed; the row sum goes to
 //               the epilogue. A row whose only visible key is itself (the -1e5
 //               self logit) is flagged: its output is v of the query itself.
-//   warps 6-9   epilogue: O from TMEM, divided by the row sum and packed to
+//   warps 9-12  epilogue: O from TMEM, divided by the row sum and packed to
 //               bf16 (the accumulator is released before the stores), staged
 //               per warp in a 4 KB swizzled buffer (32 rows x 64 columns) and
 //               written by TMA bulk stores (slot order); the softmax writes lse
@@ -60,7 +60,7 @@ namespace lsh {
 
 constexpr int kAttnM = 64;      // chunk length served by this kernel
 constexpr int kAttnKeys = 192;  // key window of a pair of chunks
-constexpr int kAttnWarps = 12;
+constexpr int kAttnWarps = 13;
 constexpr int kAttnStats = 4;   // row-sum slots between softmax and epilogue
 constexpr int kAttnRing = 4;    // metadata ring depth
 // Above this bound (log2 units) the stabiliser could push exp2 below the
@@ -68,7 +68,8 @@ constexpr int kAttnRing = 4;    // metadata ring depth
 constexpr float kAttnBoundMax = 60.f;
 
 struct AttnTcArgs {
-  const __nv_bfloat16* v;      // [BH][n][d] position order (rows that see only themselves)
+  const __nv_bfloat16* x;      // [BH][n][d] position order
+  const __nv_bfloat16* v;      // [BH][n][d] position order
   const float* pinv;           // [BH][n] 1/||x|| by position (0 for a zero row)
   const int32_t* perm;         // [S][n] position of each slot
   float* lse;                  // [S][n] each round's lse by position (the caller's output)
@@ -93,13 +94,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnWarps * 32, 1)
-    k_attn_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmo,
-              AttnTcArgs a) {
+    k_attn_tc(const __grid_constant__ CUtensorMap tmo, AttnTcArgs a) {
   using namespace sm100;
   constexpr int KH = D / 64;
   constexpr uint32_t BOX = kAttnKeys * 128;
   constexpr uint32_t TILE = KH * BOX;
-  constexpr int ROWS = kAttnKeys / 32;  // window rows per producer lane
+  constexpr int ROWS = kAttnKeys / 64;  // window rows per x-loader thread (metadata)
+  constexpr int CPR = KH * 8;            // 16-byte pieces per row
+  constexpr int RSTEP = 64 / CPR;        // rows between a loader thread's pieces
   constexpr float kLog2e = 1.4426950408889634f;
   constexpr int kNoKey = 0x7fffffff;
   extern __shared__ unsigned char smem_raw[];
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   float2* ktab = reinterpret_cast<float2*>(ostage + 4 * 32 * 128);    // [ring][192] (scale, pos)
   float* rstat = reinterpret_cast<float*>(ktab + kAttnRing * kAttnKeys);  // [4][128] 1/sum
   uint64_t* bars = reinterpret_cast<uint64_t*>(rstat + kAttnStats * 128);
-  uint64_t* xfull = bars + 0;    // [2] x rows landed (tx)
+  uint64_t* xfull = bars + 0;    // [2] x rows landed (64 x-loader threads)
   uint64_t* xfree = bars + 2;    // [2] S MMA done with the x tile
   uint64_t* vfull = bars + 4;    // [2] v rows landed (64 v-loader threads)
   uint64_t* vfree = bars + 6;    // [2] PV MMA done with the v tile
@@ -121,7 +123,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   uint64_t* ofull = bars + 14;   // PV MMA done
   uint64_t* ofree = bars + 15;   // 4 epilogue warps done reading O
   uint64_t* statf = bars + 16;   // [4] row sums written (4 softmax warps)
-  uint64_t* mfull = bars + 20;   // [ring] metadata written (32 producer lanes)
+  uint64_t* mfull = bars + 20;   // [ring] metadata written (64 x-loader threads)
   uint64_t* mfree = bars + 24;   // [ring] 4 softmax warps and 2 v-loader warps done with it
   uint64_t* drain = bars + 28;   // MMA issuer: every issued MMA has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 29);
@@ -129,12 +131,19 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   volatile int* drain_fail = reinterpret_cast<volatile int*>(bars + 31);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if ((int64_t)blockIdx.x >= a.units) return;  // uniform across the CTA
-  const int nu = (int)((a.units - 1 - blockIdx.x) / gridDim.x) + 1;
+  // this CTA's units: for every (batch, head) the run [lo, lo + cnt) of its P
+  // units; when P < G (short sequences) one run of the whole list instead
+  const int64_t P = (int64_t)a.rounds * a.pairs_per_seg, G = gridDim.x;
+  const bool per_head = P >= G;
+  const int64_t lo = per_head ? blockIdx.x * P / G : blockIdx.x * a.units / G;
+  const int64_t cnt = per_head ? (blockIdx.x + 1) * P / G - lo
+                               : (blockIdx.x + 1) * a.units / G - lo;
+  const int nu = (int)(per_head ? (a.units / P) * cnt : cnt);
+  if (nu == 0) return;  // uniform across the CTA
 
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(xfull + i, 1);
+      mbar_init(xfull + i, 64);
       mbar_init(xfree + i, 1);
       mbar_init(vfull + i, 64);
       mbar_init(vfree + i, 1);
@@ -146,7 +155,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     mbar_init(ofree, 4);
     for (int i = 0; i < kAttnStats; ++i) mbar_init(statf + i, 4);
     for (int i = 0; i < kAttnRing; ++i) {
-      mbar_init(mfull + i, 32);
+      mbar_init(mfull + i, 64);
       mbar_init(mfree + i, 4 + 2);
     }
     mbar_init(drain, 1);
@@ -154,7 +163,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     *drain_fail = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  if (warp == 4) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -168,33 +177,50 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   };
   // (batch-head, segment, first chunk) of this CTA's unit i
   auto unit_of = [&](int i, int64_t& bh, int64_t& seg, int& c0) {
-    const int64_t u = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
-    const int64_t per_bh = (int64_t)a.pairs_per_seg * a.rounds;
-    bh = u / per_bh;
-    const int rem = (int)(u - bh * per_bh);
-    const int pair = rem / a.rounds;
-    seg = bh * a.rounds + (rem - pair * a.rounds);
-    c0 = 2 * pair;
+    int64_t q;
+    if (per_head) {
+      bh = i / cnt;
+      q = lo + i % cnt;
+    } else {
+      const int64_t g = lo + i;
+      bh = g / P;
+      q = g - bh * P;
+    }
+    const int r = (int)(q / a.pairs_per_seg);
+    seg = bh * a.rounds + r;
+    c0 = 2 * (int)(q - (int64_t)r * a.pairs_per_seg);
+  };
+  // unit i's first 64 window rows are unit i - 1's last 64
+  auto carries = [&](int i) {
+    if (i == 0) return false;
+    int64_t bh, seg, bh1, seg1;
+    int c0, c01;
+    unit_of(i, bh, seg, c0);
+    unit_of(i - 1, bh1, seg1, c01);
+    return seg == seg1 && c0 == c01 + 2;
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&tmx);
-    }
-    const int oob = (int)(a.units / a.rounds / a.pairs_per_seg) * a.n;  // rows: a row past them
-    // positions (perm) of a unit's window rows lane + 32 t, and their logit
-    // scales (1/||x|| c); the loads are issued two units (perm) and one unit
-    // (norms) before the values are used
+  if (warp < 4) {
+    // ------------------------------------------------------------ loaders
+    const bool xl = warp < 2;      // x loaders also write the ring
+    const int lt = tid & 63;       // rank among this loader pair of warps
+    const unsigned char* src0 = reinterpret_cast<const unsigned char*>(xl ? a.x : a.v);
+    unsigned char* tiles = xl ? xt : vt;
+    uint64_t* full = xl ? xfull : vfull;
+    uint64_t* tfree = xl ? xfree : vfree;
+    const int piece = lt % CPR;    // this thread's 16-byte piece of every row it copies
+    const int kh = piece >> 3, cc = piece & 7;
+    // x loaders: positions (perm) of the window rows lt + 64 t of unit i and
+    // their logit scales (1/||x|| c); the loads are issued two units (perm)
+    // and one unit (norms) before the values are used
     auto perm_of = [&](int i, int (&p)[ROWS]) {
       int64_t bh, seg;
       int c0;
-      unit_of(i, bh, seg, c0);
-      const int k0 = (c0 - 1) * kAttnM;
+      if (i < nu) unit_of(i, bh, seg, c0);
 #pragma unroll
       for (int t = 0; t < ROWS; ++t) {
-        const int ks = k0 + lane + 32 * t;
-        p[t] = (i < nu && ks >= 0 && ks < a.n) ? __ldg(a.perm + seg * a.n + ks) : kNoKey;
+        const int ks = (i < nu) ? (c0 - 1) * kAttnM + lt + 64 * t : -1;
+        p[t] = (ks >= 0 && ks < a.n) ? __ldg(a.perm + seg * a.n + ks) : kNoKey;
       }
     };
     auto scale_of = [&](int i, const int (&p)[ROWS], float (&sc)[ROWS]) {
@@ -207,68 +233,76 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     };
     int p0[ROWS], p1[ROWS], p2[ROWS];
     float s0[ROWS], s1[ROWS];
-    perm_of(0, p0);
-    perm_of(1, p1);
-    scale_of(0, p0, s0);
-    scale_of(1, p1, s1);
-    perm_of(2, p2);
-    int lastx[2] = {-1, -1};
-    bool ok = true;
+    if (xl) {
+      perm_of(0, p0);
+      perm_of(1, p1);
+      scale_of(0, p0, s0);
+      scale_of(1, p1, s1);
+      perm_of(2, p2);
+    }
     for (int i = 0; i < nu; ++i) {
       const int s = i & 1, k = i >> 1, m = i & (kAttnRing - 1), km = i / kAttnRing;
-      // ring slot m free (the softmax of unit i - 4 is done with it), x tile s
-      // free (S of unit i - 2 computed)
-      bool got = (km == 0 || mbar_wait(mfree + m, (km - 1) & 1)) &&
-                 (k == 0 || mbar_wait(xfree + s, (k - 1) & 1));
-      if (__any_sync(0xffffffffu, !got || *abort_flag)) {
-        ok = __all_sync(0xffffffffu, got);
-        break;
+      bool got;
+      if (xl)  // ring slot m free (unit i - 4 done with it), x tile s free (S of unit i - 2)
+        got = (km == 0 || mbar_wait(mfree + m, (km - 1) & 1)) &&
+              (k == 0 || mbar_wait(tfree + s, (k - 1) & 1));
+      else     // ring slot m written for unit i, v tile s free (PV of unit i - 2)
+        got = mbar_wait(mfull + m, km & 1) && (k == 0 || mbar_wait(tfree + s, (k - 1) & 1));
+      if (!got) fail();
+      // both warps of the pair stop together (a failure anywhere sets
+      // abort_flag); the barrier also orders the pair's copies of unit i - 1
+      // (each thread has waited for its own) before they are read below
+      if (bar_sync_any(2 + (xl ? 0 : 1), 64, !got || *abort_flag)) break;
+      float2* kt = ktab + m * kAttnKeys;
+      if (xl) {
+#pragma unroll
+        for (int t = 0; t < ROWS; ++t) kt[lt + 64 * t] = make_float2(s0[t], __int_as_float(p0[t]));
+        bar_sync_any(2, 64, false);  // the pair's ring entries are written
+        mbar_arrive(mfull + m);
       }
       int64_t bh, seg;
       int c0;
       unit_of(i, bh, seg, c0);
-      float2* kt = ktab + m * kAttnKeys;
-#pragma unroll
-      for (int t = 0; t < ROWS; ++t) kt[lane + 32 * t] = make_float2(s0[t], __int_as_float(p0[t]));
-      mbar_arrive(mfull + m);
-      __syncwarp();  // the ring is read back below by other lanes
-      const int rbase = (int)(bh * a.n);
-      // rows 4 g .. 4 g + 3 of the window, for g = lane and lane + 32 (< 48)
-      auto gather = [&](const CUtensorMap* map, unsigned char* tile, uint64_t* bar) {
-        for (int g = lane; g < kAttnKeys / 4; g += 32) {
-          int r[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int pos = __float_as_int(kt[4 * g + j].y);
-            r[j] = pos == kNoKey ? oob : rbase + pos;
-          }
-#pragma unroll
-          for (int kh = 0; kh < KH; ++kh)
-            tma_gather4_2d(tile + kh * BOX + 4 * g * 128, map, bar, kh * 64, r[0], r[1], r[2], r[3]);
+      unsigned char* dst = tiles + s * TILE;
+      int row0 = 0;
+      if (carries(i)) {  // rows 0..63 = rows 128..191 of the previous tile
+        const unsigned char* prev = tiles + (s ^ 1) * TILE;
+        for (int e = lt; e < kAttnM * 8 * KH; e += 64) {
+          const int h = e / (kAttnM * 8), rc = e % (kAttnM * 8);  // 16-byte piece rc of half h
+          *reinterpret_cast<uint4*>(dst + h * BOX + rc * 16) =
+              *reinterpret_cast<const uint4*>(prev + h * BOX + 128 * 128 + rc * 16);
         }
-      };
-      if (lane == 0) mbar_expect_tx(xfull + s, TILE);
-      __syncwarp();
-      gather(&tmx, xt + s * TILE, xfull + s);
-      if (lane == 0) lastx[s] = k;
-      // the next units' metadata: norms one unit ahead, positions two
-#pragma unroll
-      for (int t = 0; t < ROWS; ++t) {
-        p0[t] = p1[t];
-        s0[t] = s1[t];
-        p1[t] = p2[t];
+        row0 = kAttnM;
       }
-      scale_of(i + 2, p1, s1);  // p1 now holds unit i + 2's positions
-      perm_of(i + 3, p2);
+      const unsigned char* rows = src0 + (bh * a.n) * (int64_t)(D * 2) + piece * 16;
+      unsigned char* dk = dst + kh * BOX;
+#pragma unroll 4
+      for (int row = row0 + lt / CPR; row < kAttnKeys; row += RSTEP) {
+        const int pos = __float_as_int(kt[row].y);
+        const bool valid = pos != kNoKey;
+        cp_async16_zfill(dk + row * 128 + ((cc ^ (row & 7)) << 4),
+                         valid ? rows + (int64_t)pos * (D * 2) : src0, valid);
+      }
+      cp_async_commit();
+      if (!xl) {  // done reading the ring slot
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mfree + m);
+      } else {  // the next units' metadata: norms one unit ahead, positions two
+#pragma unroll
+        for (int t = 0; t < ROWS; ++t) {
+          p0[t] = p1[t];
+          s0[t] = s1[t];
+          p1[t] = p2[t];
+        }
+        scale_of(i + 2, p1, s1);  // p1 now holds unit i + 2's positions
+        perm_of(i + 3, p2);
+      }
+      cp_async_wait_all();
+      fence_proxy_async_smem();  // the copies and the carried rows, for the tensor cores
+      mbar_arrive(full + s);
     }
-    if (lane == 0) {
-      if (!ok) fail();
-      // No copy may still be writing this CTA's shared memory when it exits:
-      // wait (bounded) for the last phase issued on every stage.
-      for (int s = 0; s < 2; ++s)
-        if (lastx[s] >= 0 && !mbar_wait(xfull + s, lastx[s] & 1)) *drain_fail = 1;
-    }
-  } else if (warp == 1) {
+    cp_async_wait_all();  // nothing of this thread's still writes shared memory at exit
+  } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, kAttnKeys);
@@ -315,7 +349,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       mma_commit(drain);
       if (!mbar_wait(drain, 0)) *drain_fail = 1;
     }
-  } else if (warp < 6) {
+  } else if (warp < 9) {
     // ------------------------------------------------------------ softmax
     const int q = warp & 3;       // TMEM lane quadrant
     const int row = q * 32 + lane;
@@ -414,7 +448,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         mbar_arrive(mfree + m);
       }
     }
-  } else if (warp < 10) {
+  } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -453,7 +487,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         if (inv <= 0.f)  // only the token itself is visible: its own value row
           vr = reinterpret_cast<const uint4*>(
               a.v + (bh * a.n + a.perm[seg * a.n + qs0 + lane]) * (int64_t)D);
-        unsigned char* stg = ostage + (warp - 6) * 32 * 128;
+        unsigned char* stg = ostage + (warp - 9) * 32 * 128;
 #pragma unroll
         for (int b = 0; b < D / 64; ++b) {  // 64 columns (128 bytes of bf16) per store
           if (lane == 0) bulk_wait_read_all();  // the previous store has read the buffer
@@ -478,48 +512,12 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       }
     }
     if (lane == 0) bulk_wait_all();
-  } else {
-    // ------------------------------------------------------------ v loaders
-    constexpr int CPR = KH * 8;      // 16-byte pieces per row
-    constexpr int RSTEP = 64 / CPR;  // rows between a thread's pieces
-    const int lt = tid - 10 * 32;    // 0..63
-    const int piece = lt % CPR, kh = piece >> 3, cc = piece & 7;
-    for (int i = 0; i < nu; ++i) {
-      const int s = i & 1, k = i >> 1, m = i & (kAttnRing - 1), km = i / kAttnRing;
-      // ring slot m written for unit i, v tile s free (PV of unit i - 2 done)
-      const bool got =
-          mbar_wait(mfull + m, km & 1) && (k == 0 || mbar_wait(vfree + s, (k - 1) & 1));
-      if (!got) fail();
-      // both loader warps stop together (a failure anywhere sets abort_flag)
-      if (bar_sync_any(3, 64, !got || *abort_flag)) break;
-      int64_t bh, seg;
-      int c0;
-      unit_of(i, bh, seg, c0);
-      const float2* kt = ktab + m * kAttnKeys;
-      const unsigned char* v0 = reinterpret_cast<const unsigned char*>(a.v);
-      const unsigned char* rows = v0 + (bh * a.n) * (int64_t)(D * 2) + piece * 16;
-      unsigned char* dst = vt + s * TILE + kh * BOX;
-#pragma unroll 4
-      for (int row = lt / CPR; row < kAttnKeys; row += RSTEP) {
-        const int pos = __float_as_int(kt[row].y);
-        const bool valid = pos != kNoKey;
-        cp_async16_zfill(dst + row * 128 + ((cc ^ (row & 7)) << 4),
-                         valid ? rows + (int64_t)pos * (D * 2) : v0, valid);
-      }
-      cp_async_commit();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(mfree + m);  // done reading the ring slot
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(vfull + s);
-    }
-    cp_async_wait_all();  // no copy of this thread still writes shared memory at exit
   }
   tc_fence_before();
   __syncthreads();
   // after a drain that gave up, TMEM is left allocated rather than freed
   // under a running MMA; the status word already records the timeout
-  if (warp == 1 && !*drain_fail) {
+  if (warp == 4 && !*drain_fail) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -342,13 +342,13 @@ lsh_status launch_attn_simt(const Dims& D, const void* xs, const void* vs, const
 }
 
 template <int DD, bool CAUSAL>
-lsh_status launch_attn_tc_k(const CUtensorMap& tmx, const CUtensorMap& tmo, const AttnTcArgs& a,
-                            unsigned grid, size_t smem, cudaStream_t st) {
+lsh_status launch_attn_tc_k(const CUtensorMap& tmo, const AttnTcArgs& a, unsigned grid,
+                            size_t smem, cudaStream_t st) {
   auto kern = k_attn_tc<DD, CAUSAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return LSH_ERR_CUDA;
-  kern<<<grid, kAttnWarps * 32, smem, st>>>(tmx, tmo, a);
+  kern<<<grid, kAttnWarps * 32, smem, st>>>(tmo, a);
   return last_cuda();
 }
 
@@ -356,14 +356,11 @@ lsh_status launch_attn_tc_k(const CUtensorMap& tmx, const CUtensorMap& tmo, cons
 lsh_status launch_attn_tc(const Dims& D, const void* x, const void* v, const int32_t* perm,
                           const float* pinv, void* out_r, float* lse, WsHeader* hdr,
                           cudaStream_t st) {
-  CUtensorMap tmx, tmo;
+  CUtensorMap tmo;  // each round's output rows, 32-row stores
   const uint64_t rows = (uint64_t)D.S * D.n;
-  const uint64_t prow = (uint64_t)D.BH * D.n;  // rows of x (position order)
-  // x: one-row boxes for the gathers; each round's output: 32-row stores
-  if (!make_tmap_bf16_2d(&tmx, x, D.d, prow, (uint64_t)D.d * 2, 64, 1) ||
-      !make_tmap_bf16_2d(&tmo, out_r, D.d, rows, (uint64_t)D.d * 2, 64, 32))
-    return LSH_ERR_CUDA;
+  if (!make_tmap_bf16_2d(&tmo, out_r, D.d, rows, (uint64_t)D.d * 2, 64, 32)) return LSH_ERR_CUDA;
   AttnTcArgs a;
+  a.x = static_cast<const __nv_bfloat16*>(x);
   a.v = static_cast<const __nv_bfloat16*>(v);
   a.pinv = pinv;
   a.perm = perm;
@@ -376,10 +373,10 @@ lsh_status launch_attn_tc(const Dims& D, const void* x, const void* v, const int
   const unsigned grid = (unsigned)std::min<int64_t>(a.units, sm_count());
   const size_t smem = attn_tc_smem(D.d);
   if (D.d == 64)
-    return D.causal ? launch_attn_tc_k<64, true>(tmx, tmo, a, grid, smem, st)
-                    : launch_attn_tc_k<64, false>(tmx, tmo, a, grid, smem, st);
-  return D.causal ? launch_attn_tc_k<128, true>(tmx, tmo, a, grid, smem, st)
-                  : launch_attn_tc_k<128, false>(tmx, tmo, a, grid, smem, st);
+    return D.causal ? launch_attn_tc_k<64, true>(tmo, a, grid, smem, st)
+                    : launch_attn_tc_k<64, false>(tmo, a, grid, smem, st);
+  return D.causal ? launch_attn_tc_k<128, true>(tmo, a, grid, smem, st)
+                  : launch_attn_tc_k<128, false>(tmo, a, grid, smem, st);
 }
 
 // 1/||x|| by position, when the hash has not written it.
