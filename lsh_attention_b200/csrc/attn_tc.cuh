@@ -75,7 +75,13 @@ struct AttnTcArgs {
   float* lse;                  // [S][n] each round's lse by position (the caller's output)
   WsHeader* hdr;
   int n, rounds, pairs_per_seg;
-  int64_t units;               // BH * pairs_per_seg * rounds
+  int units;                   // BH * pairs_per_seg * rounds
+};
+
+// One unit of work: a pair of chunks (first chunk c0) of segment seg =
+// (batch-head bh, round).
+struct AttnUnit {
+  int bh, seg, c0;
 };
 
 // 2^x by the hardware's approximate base-2 exponential (relative error near
@@ -132,13 +138,14 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // this CTA's units: for every (batch, head) the run [lo, lo + cnt) of its P
-  // units; when P < G (short sequences) one run of the whole list instead
-  const int64_t P = (int64_t)a.rounds * a.pairs_per_seg, G = gridDim.x;
+  // units; when P < G (short sequences) one run of the whole list instead.
+  // Unit, slot and segment numbers fit in 32 bits (segments x n < 2^31).
+  const int P = a.rounds * a.pairs_per_seg, G = gridDim.x;
   const bool per_head = P >= G;
-  const int64_t lo = per_head ? blockIdx.x * P / G : blockIdx.x * a.units / G;
-  const int64_t cnt = per_head ? (blockIdx.x + 1) * P / G - lo
-                               : (blockIdx.x + 1) * a.units / G - lo;
-  const int nu = (int)(per_head ? (a.units / P) * cnt : cnt);
+  const int lo = (int)(per_head ? (int64_t)blockIdx.x * P / G : (int64_t)blockIdx.x * a.units / G);
+  const int cnt = (int)(per_head ? (int64_t)(blockIdx.x + 1) * P / G - lo
+                                 : (int64_t)(blockIdx.x + 1) * a.units / G - lo);
+  const int nu = per_head ? (a.units / P) * cnt : cnt;
   if (nu == 0) return;  // uniform across the CTA
 
   if (tid == 0) {
@@ -175,29 +182,22 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     record_status(a.hdr, 5u /* LSH_ERR_TIMEOUT */);
     *abort_flag = 1;
   };
-  // (batch-head, segment, first chunk) of this CTA's unit i
-  auto unit_of = [&](int i, int64_t& bh, int64_t& seg, int& c0) {
-    int64_t q;
+  // this CTA's unit i (32-bit unsigned divisions)
+  auto unit_of = [&](int i) {
+    AttnUnit u;
+    int q;
     if (per_head) {
-      bh = i / cnt;
-      q = lo + i % cnt;
+      u.bh = (int)((unsigned)i / (unsigned)cnt);
+      q = lo + i - u.bh * cnt;
     } else {
-      const int64_t g = lo + i;
-      bh = g / P;
-      q = g - bh * P;
+      const int g = lo + i;
+      u.bh = (int)((unsigned)g / (unsigned)P);
+      q = g - u.bh * P;
     }
-    const int r = (int)(q / a.pairs_per_seg);
-    seg = bh * a.rounds + r;
-    c0 = 2 * (int)(q - (int64_t)r * a.pairs_per_seg);
-  };
-  // unit i's first 64 window rows are unit i - 1's last 64
-  auto carries = [&](int i) {
-    if (i == 0) return false;
-    int64_t bh, seg, bh1, seg1;
-    int c0, c01;
-    unit_of(i, bh, seg, c0);
-    unit_of(i - 1, bh1, seg1, c01);
-    return seg == seg1 && c0 == c01 + 2;
+    const int r = (int)((unsigned)q / (unsigned)a.pairs_per_seg);
+    u.seg = u.bh * a.rounds + r;
+    u.c0 = 2 * (q - r * a.pairs_per_seg);
+    return u;
   };
 
   if (warp < 4) {
@@ -210,36 +210,56 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     uint64_t* tfree = xl ? xfree : vfree;
     const int piece = lt % CPR;    // this thread's 16-byte piece of every row it copies
     const int kh = piece >> 3, cc = piece & 7;
-    // x loaders: positions (perm) of the window rows lt + 64 t of unit i and
+    // x loaders: positions (perm) of the window rows lt + 64 t of a unit and
     // their logit scales (1/||x|| c); the loads are issued two units (perm)
     // and one unit (norms) before the values are used
-    auto perm_of = [&](int i, int (&p)[ROWS]) {
-      int64_t bh, seg;
-      int c0;
-      if (i < nu) unit_of(i, bh, seg, c0);
+    auto perm_of = [&](bool live, const AttnUnit& u, int (&p)[ROWS]) {
 #pragma unroll
       for (int t = 0; t < ROWS; ++t) {
-        const int ks = (i < nu) ? (c0 - 1) * kAttnM + lt + 64 * t : -1;
-        p[t] = (ks >= 0 && ks < a.n) ? __ldg(a.perm + seg * a.n + ks) : kNoKey;
+        const int ks = live ? (u.c0 - 1) * kAttnM + lt + 64 * t : -1;
+        p[t] = (ks >= 0 && ks < a.n) ? __ldg(a.perm + (int64_t)u.seg * a.n + ks) : kNoKey;
       }
     };
-    auto scale_of = [&](int i, const int (&p)[ROWS], float (&sc)[ROWS]) {
-      int64_t bh = 0, seg;
-      int c0;
-      if (i < nu) unit_of(i, bh, seg, c0);
+    auto scale_of = [&](const AttnUnit& u, const int (&p)[ROWS], float (&sc)[ROWS]) {
 #pragma unroll
       for (int t = 0; t < ROWS; ++t)
-        sc[t] = p[t] != kNoKey ? __ldg(a.pinv + bh * a.n + p[t]) * c_scale : 0.f;
+        sc[t] = p[t] != kNoKey ? __ldg(a.pinv + (int64_t)u.bh * a.n + p[t]) * c_scale : 0.f;
     };
+    // Gather N window rows (first, first + RSTEP, ...) of this thread's piece:
+    // every position is read from the ring first, then the copies are issued
+    // back to back.
+    auto gather = [&](auto n_rows, int first, const float2* kt, unsigned char* dk,
+                      const unsigned char* rows) {
+      constexpr int N = decltype(n_rows)::value;
+      int pos[N];
+#pragma unroll
+      for (int k = 0; k < N; ++k) pos[k] = __float_as_int(kt[first + k * RSTEP].y);
+#pragma unroll
+      for (int k = 0; k < N; ++k) {
+        const int row = first + k * RSTEP;
+        const bool valid = pos[k] != kNoKey;
+        cp_async16_zfill(dk + row * 128 + ((cc ^ (row & 7)) << 4),
+                         valid ? rows + (int64_t)pos[k] * (D * 2) : src0, valid);
+      }
+    };
+    // units i - 1 .. i + 3
+    AttnUnit u_prev = unit_of(0), u_cur = u_prev, u_n1 = unit_of(1), u_n2 = unit_of(2),
+             u_n3 = unit_of(3);
     int p0[ROWS], p1[ROWS], p2[ROWS];
     float s0[ROWS], s1[ROWS];
     if (xl) {
-      perm_of(0, p0);
-      perm_of(1, p1);
-      scale_of(0, p0, s0);
-      scale_of(1, p1, s1);
-      perm_of(2, p2);
+      perm_of(true, u_cur, p0);
+      perm_of(1 < nu, u_n1, p1);
+      scale_of(u_cur, p0, s0);
+      scale_of(u_n1, p1, s1);
+      perm_of(2 < nu, u_n2, p2);
     }
+    // Unit i's copies are issued before unit i - 1's are awaited, so two
+    // tiles' gathers are in flight per loader thread; unit i - 1's tile is
+    // handed to the tensor cores (and its last 64 rows carried into unit i's
+    // tile) once they have landed.
+    const int pair_bar = 2 + (xl ? 0 : 1);
+    bool stopped = false;
     for (int i = 0; i < nu; ++i) {
       const int s = i & 1, k = i >> 1, m = i & (kAttnRing - 1), km = i / kAttnRing;
       bool got;
@@ -249,10 +269,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       else     // ring slot m written for unit i, v tile s free (PV of unit i - 2)
         got = mbar_wait(mfull + m, km & 1) && (k == 0 || mbar_wait(tfree + s, (k - 1) & 1));
       if (!got) fail();
-      // both warps of the pair stop together (a failure anywhere sets
-      // abort_flag); the barrier also orders the pair's copies of unit i - 1
-      // (each thread has waited for its own) before they are read below
-      if (bar_sync_any(2 + (xl ? 0 : 1), 64, !got || *abort_flag)) break;
+      // both warps of the pair stop together (a failure anywhere sets abort_flag)
+      if (bar_sync_any(pair_bar, 64, !got || *abort_flag)) {
+        stopped = true;
+        break;
+      }
       float2* kt = ktab + m * kAttnKeys;
       if (xl) {
 #pragma unroll
@@ -260,29 +281,14 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         bar_sync_any(2, 64, false);  // the pair's ring entries are written
         mbar_arrive(mfull + m);
       }
-      int64_t bh, seg;
-      int c0;
-      unit_of(i, bh, seg, c0);
       unsigned char* dst = tiles + s * TILE;
-      int row0 = 0;
-      if (carries(i)) {  // rows 0..63 = rows 128..191 of the previous tile
-        const unsigned char* prev = tiles + (s ^ 1) * TILE;
-        for (int e = lt; e < kAttnM * 8 * KH; e += 64) {
-          const int h = e / (kAttnM * 8), rc = e % (kAttnM * 8);  // 16-byte piece rc of half h
-          *reinterpret_cast<uint4*>(dst + h * BOX + rc * 16) =
-              *reinterpret_cast<const uint4*>(prev + h * BOX + 128 * 128 + rc * 16);
-        }
-        row0 = kAttnM;
-      }
-      const unsigned char* rows = src0 + (bh * a.n) * (int64_t)(D * 2) + piece * 16;
+      // rows 0..63 = rows 128..191 of the previous tile
+      const bool carry = i > 0 && u_cur.seg == u_prev.seg && u_cur.c0 == u_prev.c0 + 2;
+      const unsigned char* rows = src0 + (int64_t)u_cur.bh * a.n * (D * 2) + piece * 16;
       unsigned char* dk = dst + kh * BOX;
-#pragma unroll 4
-      for (int row = row0 + lt / CPR; row < kAttnKeys; row += RSTEP) {
-        const int pos = __float_as_int(kt[row].y);
-        const bool valid = pos != kNoKey;
-        cp_async16_zfill(dk + row * 128 + ((cc ^ (row & 7)) << 4),
-                         valid ? rows + (int64_t)pos * (D * 2) : src0, valid);
-      }
+      if (!carry) gather(std::integral_constant<int, kAttnM / RSTEP>{}, lt / CPR, kt, dk, rows);
+      gather(std::integral_constant<int, (kAttnKeys - kAttnM) / RSTEP>{}, kAttnM + lt / CPR, kt,
+             dk, rows);
       cp_async_commit();
       if (!xl) {  // done reading the ring slot
         __syncwarp();
@@ -294,14 +300,34 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
           s0[t] = s1[t];
           p1[t] = p2[t];
         }
-        scale_of(i + 2, p1, s1);  // p1 now holds unit i + 2's positions
-        perm_of(i + 3, p2);
+        scale_of(u_n2, p1, s1);  // p1 now holds unit i + 2's positions
+        perm_of(i + 3 < nu, u_n3, p2);
       }
-      cp_async_wait_all();
-      fence_proxy_async_smem();  // the copies and the carried rows, for the tensor cores
-      mbar_arrive(full + s);
+      if (i > 0) {
+        cp_async_wait_prev();  // this thread's copies of unit i - 1 have landed
+        if (carry) {
+          bar_sync_any(pair_bar, 64, false);  // ... and the whole pair's
+          const unsigned char* prev = tiles + (s ^ 1) * TILE;
+          for (int e = lt; e < kAttnM * 8 * KH; e += 64) {
+            const int h = e / (kAttnM * 8), rc = e % (kAttnM * 8);  // piece rc of half h
+            *reinterpret_cast<uint4*>(dst + h * BOX + rc * 16) =
+                *reinterpret_cast<const uint4*>(prev + h * BOX + 128 * 128 + rc * 16);
+          }
+        }
+        fence_proxy_async_smem();  // unit i - 1's rows (and unit i's carried ones) for the MMA
+        mbar_arrive(full + (s ^ 1));
+      }
+      u_prev = u_cur;
+      u_cur = u_n1;
+      u_n1 = u_n2;
+      u_n2 = u_n3;
+      u_n3 = unit_of(i + 4);
     }
     cp_async_wait_all();  // nothing of this thread's still writes shared memory at exit
+    if (!stopped) {  // the last unit
+      fence_proxy_async_smem();
+      mbar_arrive(full + ((nu - 1) & 1));
+    }
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -363,9 +389,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       // the four softmax warps; a failure seen by any of them stops all four
       // here, so none is left waiting at this barrier
       if (bar_sync_any(1, 128, !got || *abort_flag)) break;
-      int64_t bh, seg;
-      int c0;
-      unit_of(i, bh, seg, c0);
+      const AttnUnit u = unit_of(i);
+      const int64_t seg = u.seg;
+      const int c0 = u.c0;
       const float2* kt = ktab + m * kAttnKeys;
       const float2 me = kt[kAttnM + row];
       const int qpos = __float_as_int(me.y);
@@ -478,9 +504,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(ofree);
-      int64_t bh, seg;
-      int c0;
-      unit_of(i, bh, seg, c0);
+      const AttnUnit u = unit_of(i);
+      const int64_t bh = u.bh, seg = u.seg;
+      const int c0 = u.c0;
       const int qs0 = c0 * kAttnM + q * 32;  // first query slot of this warp
       if (qs0 < a.n) {  // n % 64 == 0: a warp's 32 rows are all valid or all not
         const uint4* vr = nullptr;

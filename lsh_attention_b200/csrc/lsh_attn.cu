@@ -369,7 +369,7 @@ lsh_status launch_attn_tc(const Dims& D, const void* x, const void* v, const int
   a.n = D.n;
   a.rounds = D.rounds;
   a.pairs_per_seg = (D.n / kAttnM + 1) / 2;
-  a.units = D.S * a.pairs_per_seg;
+  a.units = (int)(D.S * a.pairs_per_seg);  // < 2^31: S x n < 2^31 (attn_tc_supported)
   const unsigned grid = (unsigned)std::min<int64_t>(a.units, sm_count());
   const size_t smem = attn_tc_smem(D.d);
   if (D.d == 64)
