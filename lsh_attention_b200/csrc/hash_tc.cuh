@@ -18,10 +18,12 @@
 //     done, and ||x|| is summed by the warps that do not decide.
 // Exactness: the fp32 accumulation of d bf16 products is within
 // d * 2^-23 * sum_k |x_k R_kj| <= d * 2^-23 * ||x|| ||R_j|| of the exact sum,
-// whatever the order or rounding of the additions. When the top two |p| are
-// closer than four times that bound (kTieFactor), the token is queued and
-// k_hash_refine re-decides it in fp64 in the sequential order of the
-// definition, so the bucket equals the exact argmax bit for bit.
+// whatever the order or rounding of the additions. Two columns can only
+// trade places when their computed |p| are closer than the sum of their two
+// errors, so when the top two |p| are closer than twice that bound
+// (kTieFactor; ||x|| and the column norms enter it rounded up) the token is
+// queued and k_hash_refine re-decides it in fp64 in the sequential order of
+// the definition, so the bucket equals the exact argmax bit for bit.
 #pragma once
 
 #include "common.cuh"
@@ -37,7 +39,7 @@ constexpr int kHashMaxN = 16 * kHashMaxBatches * kHashEpiPerQuad;  // columns pe
 constexpr int kHashWarps = 2 + 4 * kHashEpiPerQuad;  // 0: TMA, 1: MMA, rest: epilogue
 // the norm pass of the attention forms ||x||^2 in this epilogue's order
 static_assert(kHashEpiPerQuad - 1 == kNormParts, "norm summation orders must agree");
-constexpr float kTieFactor = 4.0f;   // margin threshold / accumulation error bound
+constexpr float kTieFactor = 2.0f;   // margin threshold / accumulation error bound
 constexpr int kHashSmemBudget = 227 * 1024;
 
 struct HashTcPlan {
