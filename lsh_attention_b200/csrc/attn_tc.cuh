@@ -308,10 +308,23 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         if (carry) {
           bar_sync_any(pair_bar, 64, false);  // ... and the whole pair's
           const unsigned char* prev = tiles + (s ^ 1) * TILE;
-          for (int e = lt; e < kAttnM * 8 * KH; e += 64) {
-            const int h = e / (kAttnM * 8), rc = e % (kAttnM * 8);  // piece rc of half h
-            *reinterpret_cast<uint4*>(dst + h * BOX + rc * 16) =
-                *reinterpret_cast<const uint4*>(prev + h * BOX + 128 * 128 + rc * 16);
+          // every piece is loaded before the first is stored (8 at a time)
+          constexpr int NP = kAttnM * 8 * KH / 64;  // pieces per thread
+#pragma unroll
+          for (int g = 0; g < NP; g += 8) {
+            uint4 buf[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int e = lt + 64 * (g + j);
+              const int h = e / (kAttnM * 8), rc = e % (kAttnM * 8);  // piece rc of half h
+              buf[j] = *reinterpret_cast<const uint4*>(prev + h * BOX + 128 * 128 + rc * 16);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int e = lt + 64 * (g + j);
+              const int h = e / (kAttnM * 8), rc = e % (kAttnM * 8);
+              *reinterpret_cast<uint4*>(dst + h * BOX + rc * 16) = buf[j];
+            }
           }
         }
         fence_proxy_async_smem();  // unit i - 1's rows (and unit i's carried ones) for the MMA
