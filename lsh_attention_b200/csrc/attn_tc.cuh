@@ -212,18 +212,28 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     const int kh = piece >> 3, cc = piece & 7;
     // x loaders: positions (perm) of the window rows lt + 64 t of a unit and
     // their logit scales (1/||x|| c); the loads are issued two units (perm)
-    // and one unit (norms) before the values are used
-    auto perm_of = [&](bool live, const AttnUnit& u, int (&p)[ROWS]) {
+    // and one unit (norms) before the values go to the ring. Every load reads
+    // a valid address and its value is first used a unit later (validity
+    // comes from the slot number, which needs no load), so the loop never
+    // waits for one.
+    auto perm_of = [&](bool live, const AttnUnit& u, int (&raw)[ROWS], uint32_t& ok) {
+      ok = 0u;
 #pragma unroll
       for (int t = 0; t < ROWS; ++t) {
         const int ks = live ? (u.c0 - 1) * kAttnM + lt + 64 * t : -1;
-        p[t] = (ks >= 0 && ks < a.n) ? __ldg(a.perm + (int64_t)u.seg * a.n + ks) : kNoKey;
+        const bool in = ks >= 0 && ks < a.n;
+        ok |= (in ? 1u : 0u) << t;
+        raw[t] = __ldg(a.perm + (int64_t)u.seg * a.n + (in ? ks : 0));
       }
     };
-    auto scale_of = [&](const AttnUnit& u, const int (&p)[ROWS], float (&sc)[ROWS]) {
+    auto checked = [&](const int (&raw)[ROWS], uint32_t ok, int (&p)[ROWS]) {
+#pragma unroll
+      for (int t = 0; t < ROWS; ++t) p[t] = (ok >> t) & 1u ? raw[t] : kNoKey;
+    };
+    auto norm_of = [&](const AttnUnit& u, const int (&p)[ROWS], float (&raw)[ROWS]) {
 #pragma unroll
       for (int t = 0; t < ROWS; ++t)
-        sc[t] = p[t] != kNoKey ? __ldg(a.pinv + (int64_t)u.bh * a.n + p[t]) * c_scale : 0.f;
+        raw[t] = __ldg(a.pinv + (int64_t)u.bh * a.n + (p[t] != kNoKey ? p[t] : 0));
     };
     // Gather N window rows (first, first + RSTEP, ...) of this thread's piece:
     // every position is read from the ring first, then the copies are issued
@@ -245,14 +255,19 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     // units i - 1 .. i + 3
     AttnUnit u_prev = unit_of(0), u_cur = u_prev, u_n1 = unit_of(1), u_n2 = unit_of(2),
              u_n3 = unit_of(3);
-    int p0[ROWS], p1[ROWS], p2[ROWS];
-    float s0[ROWS], s1[ROWS];
+    // p0, p1: positions of units i, i + 1; r2: raw positions of unit i + 2;
+    // n0, n1: raw norms of units i, i + 1
+    int p0[ROWS], p1[ROWS], r2[ROWS];
+    float n0[ROWS], n1[ROWS];
+    uint32_t ok2 = 0u;
     if (xl) {
-      perm_of(true, u_cur, p0);
-      perm_of(1 < nu, u_n1, p1);
-      scale_of(u_cur, p0, s0);
-      scale_of(u_n1, p1, s1);
-      perm_of(2 < nu, u_n2, p2);
+      perm_of(true, u_cur, r2, ok2);
+      checked(r2, ok2, p0);
+      perm_of(1 < nu, u_n1, r2, ok2);
+      checked(r2, ok2, p1);
+      norm_of(u_cur, p0, n0);
+      norm_of(u_n1, p1, n1);
+      perm_of(2 < nu, u_n2, r2, ok2);
     }
     // Unit i's copies are issued before unit i - 1's are awaited, so two
     // tiles' gathers are in flight per loader thread; unit i - 1's tile is
@@ -277,7 +292,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       float2* kt = ktab + m * kAttnKeys;
       if (xl) {
 #pragma unroll
-        for (int t = 0; t < ROWS; ++t) kt[lt + 64 * t] = make_float2(s0[t], __int_as_float(p0[t]));
+        for (int t = 0; t < ROWS; ++t)
+          kt[lt + 64 * t] =
+              make_float2(p0[t] != kNoKey ? n0[t] * c_scale : 0.f, __int_as_float(p0[t]));
         bar_sync_any(2, 64, false);  // the pair's ring entries are written
         mbar_arrive(mfull + m);
       }
@@ -297,11 +314,11 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
 #pragma unroll
         for (int t = 0; t < ROWS; ++t) {
           p0[t] = p1[t];
-          s0[t] = s1[t];
-          p1[t] = p2[t];
+          n0[t] = n1[t];
         }
-        scale_of(u_n2, p1, s1);  // p1 now holds unit i + 2's positions
-        perm_of(i + 3 < nu, u_n3, p2);
+        checked(r2, ok2, p1);   // unit i + 2's positions, loaded a unit ago
+        norm_of(u_n2, p1, n1);
+        perm_of(i + 3 < nu, u_n3, r2, ok2);
       }
       if (i > 0) {
         cp_async_wait_prev();  // this thread's copies of unit i - 1 have landed
