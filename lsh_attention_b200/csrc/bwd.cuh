@@ -125,28 +125,39 @@ struct BwdArgs {
 
 constexpr int kNoPos = 0x7fffffff;
 
-// Warp 0 gathers `rows` rows of a [BH * n][D] tensor (row rbase + pos(r), or
-// a row past the tensor, which reads as zero, for kNoPos) into a swizzled
-// K-major tile [KH][rows][128 B] with TMA (tile::gather4: four rows per
-// instruction, each landing by its shared-memory address); completion is
-// counted on `bar`, whose expected bytes the caller sets.
-template <int D, typename PosFn>
-__device__ __forceinline__ void bwd_gather(unsigned char* tile, int rows, const CUtensorMap* map,
-                                           uint64_t* bar, int rbase, int oob, PosFn pos) {
-  constexpr int KH = D / 64;
-  const int lane = threadIdx.x & 31;
-  for (int g = lane; g < rows / 4; g += 32) {
-    int r[4];
+// All threads gather ROWS rows of a [BH * n][D] tensor (row rbase + pos(r);
+// zeros for kNoPos) into a swizzled K-major tile [KH][ROWS][128 B]: chunk c
+// of a row's 128-byte line goes to slot c ^ (row % 8), the layout the
+// 128-byte-swizzle descriptors read. Each thread copies one 16-byte piece of
+// every RSTEP-th row with cp.async, all positions read first.
+template <int D, int ROWS, typename PosFn>
+__device__ __forceinline__ void bwd_gather(unsigned char* tile, const __nv_bfloat16* src,
+                                           int64_t rbase, PosFn pos) {
+  constexpr int KH = D / 64, PPR = KH * 8;  // 16-byte pieces per row
+  constexpr int RSTEP = kBwdWarps * 32 / PPR;
+  constexpr int N = ROWS / RSTEP;
+  static_assert(ROWS % RSTEP == 0, "rows split evenly over the threads");
+  const int piece = threadIdx.x % PPR, kh = piece >> 3, c = piece & 7;
+  const int r0 = threadIdx.x / PPR;
+  int p[N];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int p = pos(4 * g + j);
-      r[j] = p == kNoPos ? oob : rbase + p;
-    }
+  for (int k = 0; k < N; ++k) p[k] = pos(r0 + k * RSTEP);
+  const unsigned char* s0 = reinterpret_cast<const unsigned char*>(src);
 #pragma unroll
-    for (int kh = 0; kh < KH; ++kh)
-      sm100::tma_gather4_2d(tile + kh * rows * 128 + 4 * g * 128, map, bar, kh * 64, r[0], r[1],
-                            r[2], r[3]);
+  for (int k = 0; k < N; ++k) {
+    const int row = r0 + k * RSTEP;
+    const bool valid = p[k] != kNoPos;
+    sm100::cp_async16_zfill(tile + kh * ROWS * 128 + row * 128 + ((c ^ (row & 7)) << 4),
+                            valid ? s0 + ((rbase + p[k]) * D + kh * 64 + c * 8) * 2 : s0, valid);
   }
+}
+
+// The gathers issued by this thread have landed; with a CTA barrier after
+// it, every thread's have, for the tensor cores too.
+__device__ __forceinline__ void bwd_gather_done() {
+  sm100::cp_async_commit();
+  sm100::cp_async_wait_all();
+  sm100::fence_proxy_async_smem();
 }
 
 // (batch-head, segment, first chunk) of unit u (numbered (batch, head), pair, round)
@@ -230,16 +241,14 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       }
     }
     __syncthreads();
-    if (warp == 0) {
-      if (lane == 0) mbar_expect_tx(bar_ld, (uint32_t)(KH * (2 * XBOX + GBOX)));
-      __syncwarp();
-      const int rb = (int)(bh * a.n);
+    {
+      const int64_t rb = bh * a.n;
       auto kpos = [&](int r) { return __float_as_int(kt[r].w); };
-      bwd_gather<D>(xt, 192, &tmx, bar_ld, rb, a.oob, kpos);
-      bwd_gather<D>(vt, 192, &tmv, bar_ld, rb, a.oob, kpos);
-      bwd_gather<D>(gt, 128, &tmg, bar_ld, rb, a.oob, [&](int r) { return __float_as_int(qt[r].x); });
+      bwd_gather<D, 192>(xt, a.x, rb, kpos);
+      bwd_gather<D, 192>(vt, a.v, rb, kpos);
+      bwd_gather<D, 128>(gt, a.g, rb, [&](int r) { return __float_as_int(qt[r].x); });
+      bwd_gather_done();
     }
-    if (!mbar_wait(bar_ld, it & 1)) *bad = 1;
     tc_fence_before();
     __syncthreads();
     // ---- S = Q K^T, dPraw = G_q V^T
@@ -411,16 +420,14 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       }
     }
     __syncthreads();
-    if (warp == 0) {
-      if (lane == 0) mbar_expect_tx(bar_ld, (uint32_t)(KH * (2 * XBOX + VBOX)));
-      __syncwarp();
-      const int rb = (int)(bh * a.n);
+    {
+      const int64_t rb = bh * a.n;
       auto qpos = [&](int r) { return __float_as_int(qt[r].x); };
-      bwd_gather<D>(xt, 192, &tmx, bar_ld, rb, a.oob, qpos);
-      bwd_gather<D>(vt, 128, &tmv, bar_ld, rb, a.oob, [&](int r) { return __float_as_int(kt[r].w); });
-      bwd_gather<D>(gt, 192, &tmg, bar_ld, rb, a.oob, qpos);
+      bwd_gather<D, 192>(xt, a.x, rb, qpos);
+      bwd_gather<D, 128>(vt, a.v, rb, [&](int r) { return __float_as_int(kt[r].w); });
+      bwd_gather<D, 192>(gt, a.g, rb, qpos);
+      bwd_gather_done();
     }
-    if (!mbar_wait(bar_ld, it & 1)) *bad = 1;
     tc_fence_before();
     __syncthreads();
     for (int pass = 0; pass < 2; ++pass, ++phase) {
