@@ -270,18 +270,20 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       }
       mma_commit(bar_sp);
     }
-    // ---- dS' = P (w dPraw + c) kd, over the S columns in bf16
-    if (warp < 4) {
+    // ---- dS' = P (w dPraw + c) kd, over the S columns in bf16; warps w and
+    // w + 4 share TMEM lane quadrant w and take alternate 32-column batches
+    {
       if (!mbar_wait(bar_sp, it & 1)) *bad = 1;
       tc_fence_after();
-      const int row = warp * 32 + lane;
-      const uint32_t tl = (uint32_t)(warp * 32) << 16;
+      const int wq = warp & 3, half = warp >> 2;
+      const int row = wq * 32 + lane;
+      const uint32_t tl = (uint32_t)(wq * 32) << 16;
       const float4 me = qt[row];
       const int qpos = __float_as_int(me.x);
       const float lse2 = me.y, w = me.z, c = me.w;
-      const int wlo = warp < 2 ? 0 : kAttnM;  // the row's window: keys [wlo, wlo + 128)
+      const int wlo = wq < 2 ? 0 : kAttnM;  // the row's window: keys [wlo, wlo + 128)
 #pragma unroll 1
-      for (int b = 0; b < 6; ++b) {
+      for (int b = half; b < 6; b += 2) {
         uint32_t sv[32], dv_[32];
         tmem_ld32(tmem + tl + b * 32, sv);
         tmem_ld32(tm_dp + tl + b * 32, dv_);
@@ -320,14 +322,15 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
                     kk > 0 ? 1u : 0u);
       mma_commit(bar_q);
     }
-    if (warp < 4) {
+    {  // dQ rows out: warps w and w + 4 write alternate 32-column blocks
       if (!mbar_wait(bar_q, it & 1)) *bad = 1;
       tc_fence_after();
-      const int row = warp * 32 + lane;
-      const uint32_t tl = (uint32_t)(warp * 32) << 16;
+      const int wq = warp & 3, half = warp >> 2;
+      const int row = wq * 32 + lane;
+      const uint32_t tl = (uint32_t)(wq * 32) << 16;
       const int qs = c0 * kAttnM + row;
 #pragma unroll
-      for (int b = 0; b < D / 32; ++b) {
+      for (int b = half; b < D / 32; b += 2) {
         uint32_t o[32];
         tmem_ld32(tm_dq + tl + b * 32, o);
         tmem_wait_ld();
@@ -453,17 +456,19 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
         }
         mma_commit(bar_sp);
       }
-      // ---- P w and dS' for key row j (thread), queries [q0, q0 + N)
-      if (warp < 4) {
+      // ---- P w and dS' for key row j (thread), queries [q0, q0 + N); warps
+      // w and w + 4 share lane quadrant w and take alternate 32-query batches
+      {
         if (!mbar_wait(bar_sp, phase & 1)) *bad = 1;
         tc_fence_after();
-        const int j = warp * 32 + lane;
-        const uint32_t tl = (uint32_t)(warp * 32) << 16;
+        const int wq = warp & 3, half = warp >> 2;
+        const int j = wq * 32 + lane;
+        const uint32_t tl = (uint32_t)(wq * 32) << 16;
         const float4 k = kt[j];
         const int kp = __float_as_int(k.w);
         const int kc = j / kAttnM;  // key chunk within the unit (0 or 1)
 #pragma unroll 1
-        for (int b = 0; b < N / 32; ++b) {
+        for (int b = half; b < N / 32; b += 2) {
           uint32_t sv[32], dv_[32];
           tmem_ld32(tmem + tl + b * 32, sv);
           tmem_ld32(tm_dp + tl + b * 32, dv_);
@@ -514,18 +519,19 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
         }
         mma_commit(bar_acc);
       }
-      if (warp < 4) {
-        if (!mbar_wait(bar_acc, phase & 1)) *bad = 1;
-        tc_fence_after();
-      }
+      if (!mbar_wait(bar_acc, phase & 1)) *bad = 1;
+      tc_fence_after();
       tc_fence_before();
       __syncthreads();  // S^T / dP^T columns are rewritten by the next pass
     }
-    // ---- key rows out: dv, and dx_key = G - x kinv^2 (x . G)
-    if (warp < 4) {
+    // ---- key rows out: dv, and dx_key = G - x kinv^2 (x . G); warps w and
+    // w + 4 both form x . G for lane quadrant w and write alternate 32-column
+    // blocks
+    {
       tc_fence_after();
-      const int j = warp * 32 + lane;
-      const uint32_t tl = (uint32_t)(warp * 32) << 16;
+      const int wq = warp & 3, half = warp >> 2;
+      const int j = wq * 32 + lane;
+      const uint32_t tl = (uint32_t)(wq * 32) << 16;
       const int sj = s0 + j;
       const float4 k = kt[j];
       // the key's own x row is row j of the query tile (keys are its first
@@ -551,7 +557,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       }
       const float fk = k.z * k.z * xg;
 #pragma unroll
-      for (int b = 0; b < D / 32; ++b) {
+      for (int b = half; b < D / 32; b += 2) {
         uint32_t gv[32], vv[32];
         tmem_ld32(tm_g + tl + b * 32, gv);
         tmem_ld32(tm_dv + tl + b * 32, vv);
