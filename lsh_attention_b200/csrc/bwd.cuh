@@ -218,27 +218,34 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_dp = tmem + 192, tm_dq = tmem + 384;
 
+  // Table entry tid (< 192) of a unit, loaded a unit ahead: the loads read
+  // a valid address and validity comes from the slot number.
+  float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+  bool pvalid = false;
+  auto fetch = [&](int64_t uu) {
+    if (uu >= a.units || tid >= 192) return;
+    int64_t bh_, seg_;
+    int c0_;
+    bwd_unit(a, uu, bh_, seg_, c0_);
+    const int ks = (c0_ - 1) * kAttnM + tid;
+    pvalid = ks >= 0 && ks < a.n;
+    const int64_t at = seg_ * a.n + (pvalid ? ks : 0);
+    pk = a.ktab[at];
+    pq = a.qtab[at];
+  };
+  fetch(blockIdx.x);
   int it = 0;
   for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x, ++it) {
     int64_t bh, seg;
     int c0;
     bwd_unit(a, u, bh, seg, c0);
-    const int k0 = (c0 - 1) * kAttnM;  // first key slot (may be < 0)
     const int64_t so = seg * a.n;
-    // ---- tables and rows
-    for (int j = tid; j < 192; j += blockDim.x) {
-      const int ks = k0 + j;
-      float4 t = make_float4(0.f, 0.f, 0.f, __int_as_float(kNoPos));
-      if (ks >= 0 && ks < a.n) {
-        const float4 k = a.ktab[so + ks];
-        t = make_float4(k.x, k.y, k.z, a.qtab[so + ks].x);
-      }
-      kt[j] = t;
-      if (j >= kAttnM) {
-        const int qs = k0 + j;
-        qt[j - kAttnM] = (qs < a.n) ? a.qtab[so + qs]
-                                    : make_float4(__int_as_float(kNoPos), 0.f, 0.f, 0.f);
-      }
+    // ---- tables (key slots (c0 - 1) 64 + j; the queries are j >= 64) and rows
+    if (tid < 192) {
+      kt[tid] = pvalid ? make_float4(pk.x, pk.y, pk.z, pq.x)
+                       : make_float4(0.f, 0.f, 0.f, __int_as_float(kNoPos));
+      if (tid >= kAttnM)
+        qt[tid - kAttnM] = pvalid ? pq : make_float4(__int_as_float(kNoPos), 0.f, 0.f, 0.f);
     }
     __syncthreads();
     {
@@ -247,6 +254,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       bwd_gather<D, 192>(xt, a.x, rb, kpos);
       bwd_gather<D, 192>(vt, a.v, rb, kpos);
       bwd_gather<D, 128>(gt, a.g, rb, [&](int r) { return __float_as_int(qt[r].x); });
+      fetch(u + gridDim.x);  // the next unit's tables, while this one computes
       bwd_gather_done();
     }
     tc_fence_before();
@@ -404,23 +412,34 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_dp = tmem + 128, tm_dv = tmem + 256, tm_g = tmem + 384;
 
+  // Table entry tid (< 192) of a unit, loaded a unit ahead: the loads read
+  // a valid address and validity comes from the slot number.
+  float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+  bool pvalid = false;
+  auto fetch = [&](int64_t uu) {
+    if (uu >= a.units || tid >= 192) return;
+    int64_t bh_, seg_;
+    int c0_;
+    bwd_unit(a, uu, bh_, seg_, c0_);
+    const int s = c0_ * kAttnM + tid;
+    pvalid = s < a.n;
+    const int64_t at = seg_ * a.n + (pvalid ? s : 0);
+    pq = a.qtab[at];
+    pk = a.ktab[at];
+  };
+  fetch(blockIdx.x);
   int phase = 0;  // completions of bar_sp and bar_acc so far (twice per unit)
-  int it = 0;     // units so far (bar_ld completes once per unit)
-  for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x, ++it) {
+  for (int64_t u = blockIdx.x; u < a.units; u += gridDim.x) {
     int64_t bh, seg;
     int c0;
     bwd_unit(a, u, bh, seg, c0);
     const int s0 = c0 * kAttnM;  // first key slot and first query slot
     const int64_t so = seg * a.n;
-    for (int j = tid; j < 192; j += blockDim.x) {
-      const int s = s0 + j;
-      const bool valid = s < a.n;
-      const float4 q = valid ? a.qtab[so + s] : make_float4(__int_as_float(kNoPos), 0.f, 0.f, 0.f);
-      qt[j] = q;
-      if (j < 128) {
-        const float4 k = valid ? a.ktab[so + s] : make_float4(0.f, 0.f, 0.f, 0.f);
-        kt[j] = make_float4(k.x, k.y, k.z, q.x);
-      }
+    if (tid < 192) {  // queries s0 + j; the keys are j < 128
+      const float4 q = pvalid ? pq : make_float4(__int_as_float(kNoPos), 0.f, 0.f, 0.f);
+      qt[tid] = q;
+      if (tid < 128)
+        kt[tid] = pvalid ? make_float4(pk.x, pk.y, pk.z, q.x) : make_float4(0.f, 0.f, 0.f, q.x);
     }
     __syncthreads();
     {
@@ -429,6 +448,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       bwd_gather<D, 192>(xt, a.x, rb, qpos);
       bwd_gather<D, 128>(vt, a.v, rb, [&](int r) { return __float_as_int(kt[r].w); });
       bwd_gather<D, 192>(gt, a.g, rb, qpos);
+      fetch(u + gridDim.x);  // the next unit's tables, while this one computes
       bwd_gather_done();
     }
     tc_fence_before();
