@@ -83,33 +83,46 @@ inline HashTcPlan hash_tc_plan(int d, int nb, int rounds) {
 // R [rounds][d][half] -> Rt [rounds][ch * nc][d]: K-major rows for the MMA's
 // B operand, each round padded with zero rows to whole chunks of nc. Also,
 // per round, an upper bound of max_j ||R_j|| (float bits in rnorm_bits[r],
-// zeroed before the launch). A CTA transposes 32 columns through shared
-// memory. grid (ceil(ch * nc / 32), rounds), block 256.
+// zeroed before the launch). A CTA transposes kPrepCols columns through
+// shared memory: a warp per column sums its squares in fp64 (rounded up at
+// the end, so any summation order gives an upper bound), and each output row
+// leaves as 16-byte stores. grid (ceil(ch * nc / kPrepCols), rounds), block
+// 256; d <= 128.
+constexpr int kPrepCols = 8;
 __global__ void __launch_bounds__(256)
     k_hash_prep(const __nv_bfloat16* __restrict__ R, __nv_bfloat16* __restrict__ Rt,
                 uint32_t* __restrict__ rnorm_bits, int d, int half, int rows_per_round) {
-  __shared__ __nv_bfloat16 tile[128][34];  // [k][column], padded rows
+  __shared__ __align__(16) __nv_bfloat16 tile[kPrepCols][128 + 8];  // [column][k]
   const int r = blockIdx.y;
-  const int j0 = blockIdx.x * 32;
+  const int j0 = blockIdx.x * kPrepCols;
   const __nv_bfloat16* src = R + (int64_t)r * d * half;
-  for (int e = threadIdx.x; e < d * 32; e += blockDim.x) {
-    const int k = e >> 5, jj = e & 31;
-    tile[k][jj] = (j0 + jj < half) ? src[(int64_t)k * half + j0 + jj] : __float2bfloat16_rn(0.f);
+  for (int e = threadIdx.x; e < d * kPrepCols; e += blockDim.x) {
+    const int k = e / kPrepCols, jj = e % kPrepCols;
+    tile[jj][k] = (j0 + jj < half) ? src[(int64_t)k * half + j0 + jj] : __float2bfloat16_rn(0.f);
   }
   __syncthreads();
-  if (threadIdx.x < 32 && j0 + threadIdx.x < half) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < kPrepCols && j0 + warp < half) {
     double ss = 0.0;
-    for (int k = 0; k < d; ++k) {
-      const double f = (double)__bfloat162float(tile[k][threadIdx.x]);
+    for (int k = lane; k < d; k += 32) {
+      const double f = (double)__bfloat162float(tile[warp][k]);
       ss += f * f;
     }
-    const float nrm = __double2float_ru(sqrt(ss));  // rounded up: an upper bound
-    atomicMax(rnorm_bits + r, __float_as_uint(nrm));  // non-negative floats order as uints
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) {
+      const float nrm = __double2float_ru(sqrt(ss));  // rounded up: an upper bound
+      atomicMax(rnorm_bits + r, __float_as_uint(nrm));  // non-negative floats order as uints
+    }
   }
+  // row jj of the output: d / 8 pieces of 16 bytes
+  const int pieces = d / 8;
   __nv_bfloat16* dst = Rt + ((int64_t)r * rows_per_round + j0) * d;
-  for (int e = threadIdx.x; e < d * 32; e += blockDim.x) {
-    const int jj = e / d, k = e % d;
-    if (j0 + jj < rows_per_round) dst[(int64_t)jj * d + k] = tile[k][jj];
+  for (int e = threadIdx.x; e < kPrepCols * pieces; e += blockDim.x) {
+    const int jj = e / pieces, c = e % pieces;
+    if (j0 + jj < rows_per_round)
+      *reinterpret_cast<uint4*>(dst + (int64_t)jj * d + c * 8) =
+          *reinterpret_cast<const uint4*>(&tile[jj][c * 8]);
   }
 }
 

@@ -204,7 +204,7 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
   __nv_bfloat16* rt = at<__nv_bfloat16>(ws, L.rt);
   uint64_t* refine = at<uint64_t>(ws, L.refine);
   const int rows_per_round = p.ch * p.nc;
-  dim3 pg((rows_per_round + 31) / 32, D.rounds);
+  dim3 pg((rows_per_round + kPrepCols - 1) / kPrepCols, D.rounds);
   k_hash_prep<<<pg, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(R), rt, hdr->pad, D.d, p.half,
                                   rows_per_round);
   if ((s = mark(ev, 1, st)) != LSH_OK) return s;
