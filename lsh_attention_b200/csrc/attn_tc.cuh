@@ -241,15 +241,19 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     auto gather = [&](auto n_rows, int first, const float2* kt, unsigned char* dk,
                       const unsigned char* rows) {
       constexpr int N = decltype(n_rows)::value;
-      int pos[N];
+      constexpr int B = N < 8 ? N : 8;  // rows per batch (keeps the code small)
+#pragma unroll 1
+      for (int g = 0; g < N; g += B) {
+        int pos[B];
 #pragma unroll
-      for (int k = 0; k < N; ++k) pos[k] = __float_as_int(kt[first + k * RSTEP].y);
+        for (int k = 0; k < B; ++k) pos[k] = __float_as_int(kt[first + (g + k) * RSTEP].y);
 #pragma unroll
-      for (int k = 0; k < N; ++k) {
-        const int row = first + k * RSTEP;
-        const bool valid = pos[k] != kNoKey;
-        cp_async16_zfill(dk + row * 128 + ((cc ^ (row & 7)) << 4),
-                         valid ? rows + (int64_t)pos[k] * (D * 2) : src0, valid);
+        for (int k = 0; k < B; ++k) {
+          const int row = first + (g + k) * RSTEP;
+          const bool valid = pos[k] != kNoKey;
+          cp_async16_zfill(dk + row * 128 + ((cc ^ (row & 7)) << 4),
+                           valid ? rows + (int64_t)pos[k] * (D * 2) : src0, valid);
+        }
       }
     };
     // units i - 1 .. i + 3
