@@ -55,17 +55,17 @@ EXTRA_WORKLOADS = ("image-12k", "bf16-short", "sweep-n131072-r8-iso", "sweep-n20
 NCU_WORKLOAD = I.LONG_64K.name
 NCU_TRAFFIC: dict = {
     "hash_mma": {"file": "hash_tc.cuh", "bytes": 152413696,
-                 "sha256": "9efe157cc7584ba239313d90470bd57910fa16c801ff4259f6a705b3a6490050"},
-    "chunk_attention": {"file": "attn_tc.cuh", "bytes": 866181632,
-                 "sha256": "e8eb44577c1141e6765d68ae41c9b5254ac42f1c2ec676ac97b892f95470b26c"},
+                 "sha256": "873d87beb4cb453dcaee820e06cfde7634041690c6f2ec915098b1569109aaba"},
+    "chunk_attention": {"file": "attn_tc.cuh", "bytes": 838573568,
+                 "sha256": "1e37f006eaa651e55be3ac720d1c9fc5d42506a6510905e847f7b9470872405a"},
     "unsort_merge": {"file": "merge.cuh", "bytes": 672992256,
                  "sha256": "f313dd4622da3353060cb7b84324a099bfef2be35a4e693135b8674f34cd17db"},
     "hash_refine": {"file": "hash_tc.cuh", "bytes": 1661184,
-                 "sha256": "9efe157cc7584ba239313d90470bd57910fa16c801ff4259f6a705b3a6490050"},
+                 "sha256": "873d87beb4cb453dcaee820e06cfde7634041690c6f2ec915098b1569109aaba"},
     "sort_rank": {"file": "sort.cuh", "bytes": 12599296,
                  "sha256": "e031792086f8fef697f441014adf16e9a9b36d922f1a623610bc2e5e46c4b5ab"},
-    "hash_prep": {"file": "hash_tc.cuh", "bytes": 531968,
-                 "sha256": "9efe157cc7584ba239313d90470bd57910fa16c801ff4259f6a705b3a6490050"},
+    "hash_prep": {"file": "hash_tc.cuh", "bytes": 533504,
+                 "sha256": "873d87beb4cb453dcaee820e06cfde7634041690c6f2ec915098b1569109aaba"},
     "sort_scan": {"file": "sort.cuh", "bytes": 4203776,
                  "sha256": "e031792086f8fef697f441014adf16e9a9b36d922f1a623610bc2e5e46c4b5ab"},
 }
