@@ -101,3 +101,26 @@ def test_backward_rejects_unsupported():
     with pytest.raises(lb.LshAttnError) as e:
         lb.lsh_attn_backward(xg, vg, bk, out, lse, out, n_buckets=8, chunk=64, causal=True)
     assert e.value.status == 2
+
+
+def test_backward_full_size_one_head():
+    """The long-64k workload (B1 H8 n65536 d128 nb1024 m64 R4, causal) in the
+    launch configuration the benchmark times; head 0's gradients against the
+    oracle, which differentiates that head alone (the heads are independent).
+    Bucket ids are the seeded synthetic ones (an input of the backward)."""
+    w = I.LONG_64K
+    x, v = I.make_qkv(w)
+    bk = I.make_buckets(w)
+    g = torch.Generator().manual_seed(5)
+    dout = torch.randn(x.shape, generator=g).to(torch.bfloat16)
+    kw = dict(n_buckets=w.n_buckets, chunk=w.chunk, causal=w.causal)
+    xg, vg, bkg = x.cuda(), v.cuda(), bk.cuda()
+    out, lse = lb.lsh_attn_forward(xg, vg, None, buckets=bkg, **kw)
+    dx, dv = lb.lsh_attn_backward(xg, vg, bkg, out, lse, dout.cuda(), **kw)
+    torch.cuda.synchronize()
+    dx0, dv0 = dx[:, :1].cpu(), dv[:, :1].cpu()
+    del xg, vg, bkg, out, lse, dx, dv
+    ref_dx, ref_dv = ob.backward(x[:, :1], v[:, :1], bk[:, :1], w.chunk, w.causal,
+                                 dout[:, :1].double(), None)
+    check_grad(dx0, ref_dx, "long-64k head 0 dx")
+    check_grad(dv0, ref_dv, "long-64k head 0 dv")

@@ -95,3 +95,22 @@ def test_rev_hashed_buckets_are_the_layers_own():
     b1, b2, _ = lb.lsh_rev_block(x1.cuda(), x2.cuda(), Wg, buckets=bk, **kw)
     assert torch.equal(a1, b1) and torch.equal(a2, b2)
     assert 0 <= int(bk.min()) and int(bk.max()) < nb
+
+
+def test_rev_full_size_matches_oracle():
+    """The layer the benchmark times (B1 n16384, 8 heads of 128, d_ff 4096,
+    4 rounds, nb 256, feed-forward chunk 4096), against the oracle, then its
+    inverse against the input."""
+    B, n, H, dh, dff, rounds, nb, fc = 1, 16384, 8, 128, 4096, 4, 256, 4096
+    W, x1, x2, bk = setup(B, n, H, dh, dff, rounds, nb)
+    Wg = {k: v.cuda() for k, v in W.items()}
+    kw = dict(heads=H, n_buckets=nb, rounds=rounds, causal=True, ffn_chunk=fc, buckets=bk.cuda())
+    y1, y2, _ = lb.lsh_rev_block(x1.cuda(), x2.cuda(), Wg, **kw)
+    y1, y2 = y1.clone(), y2.clone()
+    z1, z2, _ = lb.lsh_rev_block(y1, y2, Wg, inverse=True, **kw)
+    r1, r2 = rv.block(x1, x2, {k: v.double().numpy() for k, v in W.items()}, bk.numpy(), H, 64,
+                      True, fc)
+    check(y1, r1, "full-size y1")
+    check(y2, r2, "full-size y2")
+    check(z1, x1.double().numpy(), "full-size x1 back")
+    check(z2, x2.double().numpy(), "full-size x2 back")
