@@ -42,8 +42,11 @@
 // elementwise step, MMAs, write-out); TMEM holds [0, 512) for one unit.
 #pragma once
 
+#include <type_traits>
+
 #include "attn_tc.cuh"
 #include "common.cuh"
+#include "merge.cuh"
 #include "sm100.cuh"
 
 namespace lsh {
@@ -52,33 +55,47 @@ constexpr int kBwdWarps = 8;  // warps 0-3 own TMEM lane quadrants; all 8 load
 constexpr float kBwdLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------------------
-// grid-stride over (bh, position); block 256, one warp per position.
-// lse [BH][R][n] (natural log), out, g [BH][n][D] in T; pos_tab [BH][n]
-// float2 (LSE, g . out).
+// grid-stride over (bh, position); block 256, D * sizeof(T) / 16 lanes per
+// position. lse [BH][R][n] (natural log), out, g [BH][n][D] in T; pos_tab
+// [BH][n] float2 (LSE, g . out).
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
     k_bwd_prep_pos(const float* __restrict__ lse, const T* __restrict__ out,
                    const T* __restrict__ g, float2* __restrict__ pos_tab, int n, int rounds,
                    int64_t total) {
-  constexpr int PER = D / 32;
-  const int lane = threadIdx.x & 31;
-  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < total;
-       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-    const int64_t bh = r / n;
-    const int i = (int)(r - bh * n);
-    float dot = 0.f;
+  // a group of G lanes per position, lane j of the group one 16-byte piece of
+  // the rows of g and out
+  constexpr int G = D * (int)sizeof(T) / 16;
+  constexpr int EPV = 16 / (int)sizeof(T);
+  const int lane = threadIdx.x & 31, gl = lane % G;
+  const int64_t stride = (int64_t)gridDim.x * (blockDim.x / 32) * (32 / G);
+  const int64_t first = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * (32 / G) + lane / G;
+  // the same count for every lane: all of a warp's lanes run every shuffle
+  const int64_t iters = (total + stride - 1) / stride;
+  for (int64_t it = 0; it < iters; ++it) {
+    const int64_t r = first + it * stride;
+    const bool valid = r < total;
+    float dot = 0.f, mx = -INFINITY;
+    int bh = 0, i = 0;
+    if (valid) {
+      bh = (int)(r / n);  // BH * n < 2^31
+      i = (int)(r - (int64_t)bh * n);
+      const uint4 ga = *reinterpret_cast<const uint4*>(g + r * D + gl * EPV);
+      const uint4 oa = *reinterpret_cast<const uint4*>(out + r * D + gl * EPV);
+      float fg[EPV], fo[EPV];
+      unpack16<T>(ga, fg);
+      unpack16<T>(oa, fo);
 #pragma unroll
-    for (int k = 0; k < PER; ++k)
-      dot = fmaf(Elem<T>::to_f(g[r * D + lane + 32 * k]), Elem<T>::to_f(out[r * D + lane + 32 * k]),
-                 dot);
-    dot = warp_sum(dot);
-    float mx = -INFINITY;
-    for (int q = lane; q < rounds; q += 32) mx = fmaxf(mx, lse[(bh * rounds + q) * n + i]);
-    mx = warp_max(mx);
+      for (int e = 0; e < EPV; ++e) dot = fmaf(fg[e], fo[e], dot);
+      for (int q = gl; q < rounds; q += G) mx = fmaxf(mx, lse[((int64_t)bh * rounds + q) * n + i]);
+    }
+    dot = group_sum<G>(dot);
+    mx = group_max<G>(mx);
     float z = 0.f;
-    for (int q = lane; q < rounds; q += 32) z += expf(lse[(bh * rounds + q) * n + i] - mx);
-    z = warp_sum(z);
-    if (lane == 0) pos_tab[r] = make_float2(mx + logf(z), dot);
+    if (valid)
+      for (int q = gl; q < rounds; q += G) z += expf(lse[((int64_t)bh * rounds + q) * n + i] - mx);
+    z = group_sum<G>(z);
+    if (valid && gl == 0) pos_tab[r] = make_float2(mx + logf(z), dot);
   }
 }
 
@@ -618,35 +635,59 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
 }
 
 // ---------------------------------------------------------------------------
-// grid-stride over (bh, position), a warp per position (d / 32 elements per
-// lane): sums the query and key roles of every round through inv.
+// grid-stride over (bh, position), a warp per position, lane j owning the
+// d / 32 consecutive elements from (d / 32) j: sums the query and key roles of
+// every round through inv, in round order. The slots of every round are
+// loaded first (one lane per round), then the rows of up to four rounds at a
+// time, all in flight together.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
     k_bwd_unsort(const int32_t* __restrict__ inv, const float* __restrict__ dq,
                  const float* __restrict__ dxk, const float* __restrict__ dvs,
                  T* __restrict__ dx, T* __restrict__ dv, int n, int rounds, int64_t total) {
-  constexpr int PER = D / 32;
+  constexpr int EPL = D / 32;  // elements per lane: 2 or 4
+  using V = typename std::conditional<EPL == 4, float4, float2>::type;
+  constexpr int RB = 4;        // rounds in flight
   const int lane = threadIdx.x & 31;
+  auto vget = [](const V& a, int e) {
+    if constexpr (EPL == 4) return e == 0 ? a.x : e == 1 ? a.y : e == 2 ? a.z : a.w;
+    else return e == 0 ? a.x : a.y;
+  };
   for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < total;
        r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
     const int64_t bh = r / n;
     const int i = (int)(r - bh * n);
-    float ax[PER], av[PER];
+    const int my_slot = lane < rounds ? inv[(bh * rounds + lane) * n + i] : 0;
+    float ax[EPL], av[EPL];
 #pragma unroll
-    for (int k = 0; k < PER; ++k) ax[k] = av[k] = 0.f;
-    for (int q = 0; q < rounds; ++q) {
-      const int64_t seg = bh * rounds + q;
-      const int64_t row = (seg * n + inv[seg * n + i]) * D;
+    for (int e = 0; e < EPL; ++e) ax[e] = av[e] = 0.f;
+    for (int q0 = 0; q0 < rounds; q0 += RB) {
+      V a[RB], b[RB], c[RB];
 #pragma unroll
-      for (int k = 0; k < PER; ++k) {
-        ax[k] += dq[row + lane + 32 * k] + dxk[row + lane + 32 * k];
-        av[k] += dvs[row + lane + 32 * k];
+      for (int t = 0; t < RB; ++t) {
+        const int q = q0 + t;
+        const int slot = __shfl_sync(0xffffffffu, my_slot, q & 31);
+        if (q < rounds) {
+          const int64_t row = ((bh * rounds + q) * n + slot) * D + lane * EPL;
+          a[t] = *reinterpret_cast<const V*>(dq + row);
+          b[t] = *reinterpret_cast<const V*>(dxk + row);
+          c[t] = *reinterpret_cast<const V*>(dvs + row);
+        }
       }
+#pragma unroll
+      for (int t = 0; t < RB; ++t)
+        if (q0 + t < rounds) {
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) {
+            ax[e] += vget(a[t], e) + vget(b[t], e);
+            av[e] += vget(c[t], e);
+          }
+        }
     }
 #pragma unroll
-    for (int k = 0; k < PER; ++k) {
-      dx[r * D + lane + 32 * k] = Elem<T>::from_f(ax[k]);
-      dv[r * D + lane + 32 * k] = Elem<T>::from_f(av[k]);
+    for (int e = 0; e < EPL; ++e) {
+      dx[r * D + lane * EPL + e] = Elem<T>::from_f(ax[e]);
+      dv[r * D + lane * EPL + e] = Elem<T>::from_f(av[e]);
     }
   }
 }

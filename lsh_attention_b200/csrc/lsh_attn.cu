@@ -612,7 +612,10 @@ lsh_status backward_d(const Dims& D, const BwdLayout& L, const void* x, const vo
   const int sms = sm_count();
   const int64_t pos_total = D.BH * D.n;
   float2* pos_tab = at<float2>(ws, L.pos_tab);
-  k_bwd_prep_pos<T, DD><<<(unsigned)std::min<int64_t>((pos_total + 7) / 8, 8 * sms), 256, 0, st>>>(
+  const int64_t pos_per_block = 8 * (32 / (DD * (int)sizeof(T) / 16));
+  k_bwd_prep_pos<T, DD><<<(unsigned)std::min<int64_t>((pos_total + pos_per_block - 1) / pos_per_block,
+                                                      8 * sms),
+                          256, 0, st>>>(
       lse, static_cast<const T*>(out), static_cast<const T*>(dout), pos_tab, D.n, D.rounds,
       pos_total);
   const int64_t slot_total = D.S * D.n;
