@@ -562,14 +562,15 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       __syncthreads();  // S^T / dP^T columns are rewritten by the next pass
     }
     // ---- key rows out: dv, and dx_key = G - x kinv^2 (x . G); warps w and
-    // w + 4 both form x . G for lane quadrant w and write alternate 32-column
-    // blocks
+    // w + 4 both form x . G for lane quadrant w and each write one half of the
+    // columns. A warp stages its 32 rows of a half in shared memory (the v and
+    // g tiles are free now) and writes them row by row, so the global stores
+    // are whole contiguous runs.
     {
       tc_fence_after();
       const int wq = warp & 3, half = warp >> 2;
       const int j = wq * 32 + lane;
       const uint32_t tl = (uint32_t)(wq * 32) << 16;
-      const int sj = s0 + j;
       const float4 k = kt[j];
       // the key's own x row is row j of the query tile (keys are its first
       // 128 rows): 16-byte chunk c of each 64-column half at slot c ^ (j % 8)
@@ -593,33 +594,47 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
         }
       }
       const float fk = k.z * k.z * xg;
+      constexpr int CW = D / 2;     // columns of a half
+      constexpr int RS = CW + 4;    // staged row stride in floats (conflict-free)
+      constexpr int LPR = CW / 4;   // lanes per row when writing out
+      constexpr int RPI = 32 / LPR; // rows per write instruction
+      float* stg = reinterpret_cast<float*>(vt) + warp * 32 * RS;
+      // which = 0: dx_key, 1: dv
+      for (int which = 0; which < 2; ++which) {
 #pragma unroll
-      for (int b = half; b < D / 32; b += 2) {
-        uint32_t gv[32], vv[32];
-        tmem_ld32(tm_g + tl + b * 32, gv);
-        tmem_ld32(tm_dv + tl + b * 32, vv);
-        tmem_wait_ld();
-        if (sj < a.n) {
-          float4* dx = reinterpret_cast<float4*>(a.dxk + (so + sj) * D + b * 32);
-          float4* dvv = reinterpret_cast<float4*>(a.dv + (so + sj) * D + b * 32);
+        for (int bb = 0; bb < CW / 32; ++bb) {
+          const int b = half * (CW / 32) + bb;
+          uint32_t tv[32];
+          tmem_ld32((which == 0 ? tm_g : tm_dv) + tl + b * 32, tv);
+          tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            float f[8];
-            xrow8(b * 4 + q, f);
-            dx[2 * q] = make_float4(__uint_as_float(gv[8 * q]) - f[0] * fk,
-                                    __uint_as_float(gv[8 * q + 1]) - f[1] * fk,
-                                    __uint_as_float(gv[8 * q + 2]) - f[2] * fk,
-                                    __uint_as_float(gv[8 * q + 3]) - f[3] * fk);
-            dx[2 * q + 1] = make_float4(__uint_as_float(gv[8 * q + 4]) - f[4] * fk,
-                                        __uint_as_float(gv[8 * q + 5]) - f[5] * fk,
-                                        __uint_as_float(gv[8 * q + 6]) - f[6] * fk,
-                                        __uint_as_float(gv[8 * q + 7]) - f[7] * fk);
-          }
+            float o[8];
+            if (which == 0) {
+              float f[8];
+              xrow8(b * 4 + q, f);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dvv[q] = make_float4(__uint_as_float(vv[4 * q]), __uint_as_float(vv[4 * q + 1]),
-                                 __uint_as_float(vv[4 * q + 2]), __uint_as_float(vv[4 * q + 3]));
+              for (int e = 0; e < 8; ++e) o[e] = __uint_as_float(tv[8 * q + e]) - f[e] * fk;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) o[e] = __uint_as_float(tv[8 * q + e]);
+            }
+            float4* dst = reinterpret_cast<float4*>(stg + lane * RS + bb * 32 + 8 * q);
+            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+          }
         }
+        __syncwarp();
+        float* gdst = (which == 0 ? a.dxk : a.dv) + half * CW;
+#pragma unroll 4
+        for (int r0 = 0; r0 < 32; r0 += RPI) {
+          const int rr = r0 + lane / LPR, c4 = lane % LPR;
+          const int sj = s0 + wq * 32 + rr;
+          if (sj < a.n)
+            *reinterpret_cast<float4*>(gdst + (so + sj) * D + c4 * 4) =
+                *reinterpret_cast<const float4*>(stg + rr * RS + c4 * 4);
+        }
+        __syncwarp();  // the staging rows are rewritten by the next array
       }
     }
     tc_fence_before();
