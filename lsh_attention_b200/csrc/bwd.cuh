@@ -347,25 +347,37 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
                     kk > 0 ? 1u : 0u);
       mma_commit(bar_q);
     }
-    {  // dQ rows out: warps w and w + 4 write alternate 32-column blocks
+    {  // dQ rows out: warps w and w + 4 each write one half of the columns,
+       // staged per warp in shared memory (the v and g tiles are free) and
+       // written as contiguous row runs
       if (!mbar_wait(bar_q, it & 1)) *bad = 1;
       tc_fence_after();
       const int wq = warp & 3, half = warp >> 2;
-      const int row = wq * 32 + lane;
       const uint32_t tl = (uint32_t)(wq * 32) << 16;
-      const int qs = c0 * kAttnM + row;
+      constexpr int CW = D / 2;     // columns of a half
+      constexpr int RS = CW + 4;    // staged row stride in floats (conflict-free)
+      constexpr int LPR = CW / 4;   // lanes per row when writing out
+      constexpr int RPI = 32 / LPR; // rows per write instruction
+      float* stg = reinterpret_cast<float*>(vt) + warp * 32 * RS;
 #pragma unroll
-      for (int b = half; b < D / 32; b += 2) {
+      for (int bb = 0; bb < CW / 32; ++bb) {
         uint32_t o[32];
-        tmem_ld32(tm_dq + tl + b * 32, o);
+        tmem_ld32(tm_dq + tl + (half * (CW / 32) + bb) * 32, o);
         tmem_wait_ld();
-        if (qs < a.n) {
-          float4* dst = reinterpret_cast<float4*>(a.dq + (so + qs) * D + b * 32);
+        float4* d4 = reinterpret_cast<float4*>(stg + lane * RS + bb * 32);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            dst[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
-                                 __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
-        }
+        for (int k = 0; k < 8; ++k)
+          d4[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
+                              __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+      }
+      __syncwarp();
+#pragma unroll 4
+      for (int r0 = 0; r0 < 32; r0 += RPI) {
+        const int rr = r0 + lane / LPR, c4 = lane % LPR;
+        const int qs = c0 * kAttnM + wq * 32 + rr;
+        if (qs < a.n)
+          *reinterpret_cast<float4*>(a.dq + (so + qs) * D + half * CW + c4 * 4) =
+              *reinterpret_cast<const float4*>(stg + rr * RS + c4 * 4);
       }
     }
     tc_fence_before();
