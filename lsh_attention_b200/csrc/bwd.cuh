@@ -309,6 +309,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
       const int wlo = wq < 2 ? 0 : kAttnM;  // the row's window: keys [wlo, wlo + 128)
 #pragma unroll 1
       for (int b = half; b < 6; b += 2) {
+        if (b * 32 < wlo || b * 32 >= wlo + 128) {  // keys outside the row's window: dS' = 0
+          uint32_t z[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) z[c] = 0u;
+          tmem_st16(tmem + tl + b * 16, z);
+          continue;
+        }
         uint32_t sv[32], dv_[32];
         tmem_ld32(tmem + tl + b * 32, sv);
         tmem_ld32(tm_dp + tl + b * 32, dv_);
