@@ -32,8 +32,9 @@
 //                    into TMEM, dS' written over S in bf16, dQ = dS' X_window
 //                    (A read from TMEM); dQ rows out, fp32, slot order
 //   k_bwd_dkv        key-stationary, a pair of chunks of keys per unit (128
-//                    keys, the 192 queries that see them, in two passes of 128
-//                    and 64): S^T = K Q^T and dPraw^T = V G^T into TMEM,
+//                    keys, the 192 queries that see them, in two passes: the
+//                    middle chunk, then the first and the last): S^T = K Q^T
+//                    and dPraw^T = V G^T into TMEM,
 //                    P w and dS' written over them in bf16, dV += (P w) G_q and
 //                    G += dS' X_q (A read from TMEM); after both passes the key
 //                    rows of dx and dv out, fp32, slot order
@@ -489,31 +490,39 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
     }
     tc_fence_before();
     __syncthreads();
+    // Pass 0 takes the middle query chunk (64 queries), which both key chunks
+    // see; pass 1 the first and the last (128 queries), each of which one key
+    // chunk sees: every warp then computes one 32-query batch per pass and
+    // writes zeros for the other. Column c of a pass is query row qrow(c).
     for (int pass = 0; pass < 2; ++pass, ++phase) {
-      const int q0 = pass * 128, N = pass == 0 ? 128 : 64;  // queries [q0, q0 + N)
-      // ---- S^T = K Q^T, dPraw^T = V_k G_q^T
+      const int N = pass == 0 ? 64 : 128;
+      auto qrow = [&](int c) { return pass == 0 ? kAttnM + c : (c < kAttnM ? c : kAttnM + c); };
+      // ---- S^T = K Q^T, dPraw^T = V_k G_q^T, 64 query columns per MMA
       if (tid == 0) {
         tc_fence_after();
         const uint32_t xa = smem_u32(xt), va = smem_u32(vt), ga = smem_u32(gt);
-        const uint32_t idesc = idesc_bf16_f32(128, N);
+        const uint32_t idesc = idesc_bf16_f32(128, kAttnM);
+        for (int part = 0; part < N / kAttnM; ++part) {
+          const int r0 = qrow(part * kAttnM);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int kh = kk >> 2, ks = kk & 3;
-          mma_bf16_ss(tmem, desc_kmajor_sw128(xa + kh * XBOX + ks * 32),
-                      desc_kmajor_sw128(xa + kh * XBOX + q0 * 128 + ks * 32), idesc,
-                      kk > 0 ? 1u : 0u);
-        }
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int kh = kk >> 2, ks = kk & 3;
+            mma_bf16_ss(tmem + part * kAttnM, desc_kmajor_sw128(xa + kh * XBOX + ks * 32),
+                        desc_kmajor_sw128(xa + kh * XBOX + r0 * 128 + ks * 32), idesc,
+                        kk > 0 ? 1u : 0u);
+          }
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int kh = kk >> 2, ks = kk & 3;
-          mma_bf16_ss(tm_dp, desc_kmajor_sw128(va + kh * VBOX + ks * 32),
-                      desc_kmajor_sw128(ga + kh * XBOX + q0 * 128 + ks * 32), idesc,
-                      kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int kh = kk >> 2, ks = kk & 3;
+            mma_bf16_ss(tm_dp + part * kAttnM, desc_kmajor_sw128(va + kh * VBOX + ks * 32),
+                        desc_kmajor_sw128(ga + kh * XBOX + r0 * 128 + ks * 32), idesc,
+                        kk > 0 ? 1u : 0u);
+          }
         }
         mma_commit(bar_sp);
       }
-      // ---- P w and dS' for key row j (thread), queries [q0, q0 + N); warps
-      // w and w + 4 share lane quadrant w and take alternate 32-query batches
+      // ---- P w and dS' for key row j (thread), the pass's queries; warps w
+      // and w + 4 share lane quadrant w and take alternate 32-query batches
       {
         if (!mbar_wait(bar_sp, phase & 1)) *bad = 1;
         tc_fence_after();
@@ -525,6 +534,15 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
         const int kc = j / kAttnM;  // key chunk within the unit (0 or 1)
 #pragma unroll 1
         for (int b = half; b < N / 32; b += 2) {
+          const int qcb = qrow(b * 32) / kAttnM;  // the batch's query chunk (0, 1 or 2)
+          if (kc != qcb && kc != qcb - 1) {       // the key's chunk is outside its window
+            uint32_t z[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) z[c] = 0u;
+            tmem_st16(tmem + tl + b * 16, z);
+            tmem_st16(tm_dp + tl + b * 16, z);
+            continue;
+          }
           uint32_t sv[32], dv_[32];
           tmem_ld32(tmem + tl + b * 32, sv);
           tmem_ld32(tm_dp + tl + b * 32, dv_);
@@ -535,7 +553,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
             float ow[2], od[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int i = q0 + b * 32 + cc + h;  // query index in the unit
+              const int i = qrow(b * 32 + cc + h);  // query index in the unit
               const float4 q = qt[i];
               const int qp = __float_as_int(q.x);
               const int qc = i / kAttnM;  // query chunk within the unit (0, 1 or 2)
@@ -568,10 +586,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
         const uint32_t idesc = idesc_bf16_f32(128, D) | (1u << 16);
         for (int kk = 0; kk < N / 16; ++kk) {
           const uint32_t acc = (pass > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16_ts(tm_dv, tmem + kk * 8, desc_mnmajor_sw128(ga + (q0 + kk * 16) * 128, XBOX),
-                      idesc, acc);
-          mma_bf16_ts(tm_g, tm_dp + kk * 8, desc_mnmajor_sw128(xa + (q0 + kk * 16) * 128, XBOX),
-                      idesc, acc);
+          const int r = qrow(kk * 16);  // 16 queries of one chunk
+          mma_bf16_ts(tm_dv, tmem + kk * 8, desc_mnmajor_sw128(ga + r * 128, XBOX), idesc, acc);
+          mma_bf16_ts(tm_g, tm_dp + kk * 8, desc_mnmajor_sw128(xa + r * 128, XBOX), idesc, acc);
         }
         mma_commit(bar_acc);
       }
