@@ -327,10 +327,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
           float o2[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int j = b * 32 + cc + h;
-            const float4 k = kt[j];
+            const float4 k = kt[b * 32 + cc + h];
             const int kp = __float_as_int(k.w);
-            const bool in_window = j >= wlo && j < wlo + 128 && kp != kNoPos;
+            const bool in_window = kp != kNoPos;  // the batch lies in the row's window
             const bool live = in_window && kp != qpos && (!CAUSAL || kp < qpos);
             const float p = ex2_approx(fmaf(__uint_as_float(sv[cc + h]), k.x, -lse2));
             const float ds = p * fmaf(w, __uint_as_float(dv_[cc + h]), c) * k.y;
@@ -548,17 +547,17 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 1)
           tmem_ld32(tm_dp + tl + b * 32, dv_);
           tmem_wait_ld();
           uint32_t pw[16], pd[16];
+          const float4* qb = qt + qrow(b * 32);  // the batch's 32 queries, one chunk
+          const bool kvalid = kp != kNoPos;
 #pragma unroll
           for (int cc = 0; cc < 32; cc += 2) {
             float ow[2], od[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int i = qrow(b * 32 + cc + h);  // query index in the unit
-              const float4 q = qt[i];
+              const float4 q = qb[cc + h];
               const int qp = __float_as_int(q.x);
-              const int qc = i / kAttnM;  // query chunk within the unit (0, 1 or 2)
-              // query chunk qc sees key chunks qc - 1 and qc
-              const bool window = kp != kNoPos && qp != kNoPos && (kc == qc || kc == qc - 1);
+              // the batch's chunk sees this key's chunk (tested above)
+              const bool window = kvalid && qp != kNoPos;
               const bool self = window && kp == qp;
               const bool live = window && kp != qp && (!CAUSAL || kp < qp);
               // the self logit is -1e5: weight 1 for a row that sees only
