@@ -8,14 +8,18 @@
 //     (transposed to K-major by k_hash_prep, loaded once by TMA);
 //   * warp 0 streams 128-token tiles of x with TMA (double-buffered);
 //   * warp 1 issues tcgen05.mma (M = 128 tokens, N <= 192 columns, K = d)
-//     into one of two TMEM accumulators, so the next unit's MMA overlaps the
-//     epilogue of the current one;
+//     into a ring of TMEM accumulators (two, or four when N <= 128), so the
+//     next units' MMAs overlap the epilogue of the current one;
 //   * warps 2..13 read the fp32 projections with tcgen05.ld and keep, per
 //     token, the largest and second largest |p_j|, the argmax and its sign
 //     (three warps per TMEM lane quadrant, each on a contiguous range of at
 //     most four 16-column batches, all loaded before one wait). The
 //     accumulator is handed back to the MMA as soon as a warp's loads are
-//     done, and ||x|| is summed by the warps that do not decide.
+//     done, and ||x|| is summed by the warps that do not decide. When a
+//     round is one unit of at most 128 columns (b <= 256), the three warps of
+//     a quadrant instead take whole units in turn, each deciding its own
+//     rounds with no combine (the per-round top-two and combine would
+//     otherwise cost more than the round's columns).
 // Exactness: the fp32 accumulation of d bf16 products is within
 // d * 2^-23 * sum_k |x_k R_kj| <= d * 2^-23 * ||x|| ||R_j|| of the exact sum,
 // whatever the order or rounding of the additions. Two columns can only
@@ -48,6 +52,8 @@ struct HashTcPlan {
   int group;        // rounds resident per CTA
   int groups;       // ceil(rounds / group)
   int tmem_cols;    // per accumulator buffer (power of two >= 32)
+  int upw;          // 1: a round is one unit of <= 128 columns, taken whole by one warp
+  int stages;       // TMEM accumulators in the MMA -> epilogue ring (2, or 4 when upw)
   size_t smem;      // dynamic shared memory
   size_t x_bytes, r_bytes;
 };
@@ -75,6 +81,8 @@ inline HashTcPlan hash_tc_plan(int d, int nb, int rounds) {
   int tc = 32;
   while (tc < p.nc) tc <<= 1;
   p.tmem_cols = tc;
+  p.upw = (p.ch == 1 && p.nc <= 128) ? 1 : 0;
+  p.stages = p.upw ? 4 : 2;  // 4 x 128 columns at most: the whole TMEM
   p.smem = p.x_bytes + p.r_bytes + misc;
   return p;
 }
@@ -357,7 +365,35 @@ __device__ __forceinline__ void top2_merge(float& m1, float& m2, int& idx, float
   }
 }
 
+// One token's decision for round r: bucket id, the sort's histogram count,
+// 1/||x|| (first round), and the near-tie test. sst = ||x||^2 in the order of
+// the attention's norm pass; rn = the round's bound of max_j ||R_j||.
 template <int D>
+__device__ __forceinline__ void hash_decide(const HashTcArgs& a, const HashTcPlan& p, int bh, int t,
+                                            int r, float m1, float m2, int idx, float sv, float sst,
+                                            float rn) {
+  if (a.pinv != nullptr && r == 0)  // once per token, from the first round
+    a.pinv[(int64_t)bh * a.n + t] = sst > 0.f ? 1.0f / sqrtf(sst) : 0.f;
+  // ||x|| rounded up past the fp32 rounding of its square sum
+  const float xnorm = sqrtf(sst) * 1.0001f;
+  const float tau = kTieFactor * (float)D * 1.1920929e-7f * xnorm * rn;
+  const int bucket = idx + (sv < 0.f ? p.half : 0);
+  const int64_t at = ((int64_t)bh * a.rounds + r) * a.n + t;
+  a.buckets[at] = bucket;
+  if (a.hist != nullptr)  // the sort's tile histogram, counted here
+    atomicAdd(a.hist + ((int64_t)(bh * a.rounds + r) * a.nb + bucket) * a.sort_tiles +
+                  t / a.sort_tile,
+              1);
+  if (!(m1 - m2 > tau)) {
+    atomicAdd(&a.hdr->hash_refined, 1u);
+    const uint32_t k = atomicAdd(&a.hdr->pad[16 + r], 1u);
+    a.refine[r * a.cap + k] = (uint64_t)((int64_t)bh * a.n + t);
+  }
+}
+
+// UPW: the plan's upw, as a template parameter so that each form compiles on
+// its own.
+template <int D, bool UPW>
 __global__ void __launch_bounds__(kHashWarps * 32, 1)
     k_hash_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmr,
               HashTcArgs a, HashTcPlan p) {
@@ -373,14 +409,15 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
   uint64_t* r_full = bars + 0;
   uint64_t* x_full = bars + 1;     // [2]
   uint64_t* x_empty = bars + 3;    // [2]
-  uint64_t* acc_full = bars + 5;   // [2]
-  uint64_t* acc_empty = bars + 7;  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 10);
-  uint64_t* drain = bars + 11;  // MMA issuer: every issued MMA has completed
-  volatile int* drain_fail = reinterpret_cast<volatile int*>(bars + 12);
+  uint64_t* acc_full = bars + 5;   // [stages <= 4]
+  uint64_t* acc_empty = bars + 9;  // [stages <= 4]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
+  uint64_t* drain = bars + 15;  // MMA issuer: every issued MMA has completed
+  volatile int* drain_fail = reinterpret_cast<volatile int*>(bars + 16);
   constexpr int PO = kHashEpiPerQuad - 1;  // warps of a quadrant that report to h = 0
-  float4* comb = reinterpret_cast<float4*>(bars + 16);  // [2][4][PO][32]
+  constexpr int S = UPW ? 4 : 2;  // p.stages
+  float4* comb = reinterpret_cast<float4*>(bars + 18);  // [2][4][PO][32]
   float* ssb = reinterpret_cast<float*>(comb + 2 * 4 * PO * 32);  // [2][4][PO][32]
   float* rn_s = ssb + 2 * 4 * PO * 32;                             // [rounds <= 16]
 
@@ -394,9 +431,14 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
     mbar_init(r_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(x_full + i, 1);
-      mbar_init(x_empty + i, 1 + 4 * PO);  // MMA commit + the norm-reading warps
+      // MMA commit + the warps that read x: the norm-summing ones, or every
+      // epilogue warp when warps take whole units
+      mbar_init(x_empty + i, 1 + 4 * (UPW ? kHashEpiPerQuad : PO));
+    }
+    for (int i = 0; i < S; ++i) {
       mbar_init(acc_full + i, 1);
-      mbar_init(acc_empty + i, 4 * kHashEpiPerQuad);  // every epilogue warp
+      // every epilogue warp, or the one warp per quadrant that takes the unit
+      mbar_init(acc_empty + i, UPW ? 4 : 4 * kHashEpiPerQuad);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -405,7 +447,7 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
   }
   if (threadIdx.x < a.rounds)  // per-round bound of max_j ||R_j|| (k_hash_prep)
     rn_s[threadIdx.x] = reinterpret_cast<const float*>(a.hdr->pad)[threadIdx.x];
-  if (warp == 1) tmem_alloc(tmem_slot, 2 * p.tmem_cols);
+  if (warp == 1) tmem_alloc(tmem_slot, S * p.tmem_cols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -474,7 +516,7 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
         const uint32_t a_lo = (uint32_t)(xb ? xd1 : xd0);
         for (int rl = 0; rl < gr && ok; ++rl) {
           for (int c = 0; c < p.ch; ++c, ++u) {
-            const int ab = u & 1, uk = u >> 1;
+            const int ab = u % S, uk = u / S;
             if (uk > 0 && !mbar_wait(acc_empty + ab, (uk - 1) & 1)) { fail(); ok = false; break; }
             if (*abort_flag) { ok = false; break; }
             tc_fence_after();
@@ -498,6 +540,86 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
       // TMEM is freed below: every MMA issued must have completed first
       mma_commit(drain);
       if (!mbar_wait(drain, 0)) *drain_fail = 1;
+    }
+  } else if (UPW) {
+    // ------------------------------------------- epilogue, whole units per warp
+    // Unit u (one round of one tile) goes to warp h = u % 3 of every
+    // quadrant, which reduces all of its columns, hands the accumulator back
+    // after its last loads and decides. Every epilogue warp waits for each x
+    // tile and releases it; a warp with a unit of the tile first sums
+    // ||x_row||^2 in the attention's norm-pass order (piece cc into part
+    // cc % kNormParts, then 0 + part_0 + part_1 + ...).
+    const int e = warp - 2;
+    const int q = warp & 3;
+    const int h = e >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t tlane = (uint32_t)(q * 32) << 16;
+    const int nbc = (p.half + 15) >> 4;  // 16-column batches of a round
+    int it = 0, u = 0;
+    bool ok = true;
+    for (int tile = li; ok && tile < a.tiles; tile += a.ctas_per_group, ++it) {
+      const int xb = it & 1, xk = it >> 1;
+      const int bh = tile / a.tiles_per_seq;
+      const int t = (tile % a.tiles_per_seq) * kHashTile + row;
+      // this tile's units are u .. u + gr - 1; this warp's first is at offset
+      const int first = (h - u % kHashEpiPerQuad + kHashEpiPerQuad) % kHashEpiPerQuad;
+      if (!mbar_wait(x_full + xb, xk & 1)) {
+        fail();
+        break;
+      }
+      float sst = 0.f;
+      if (first < gr) {
+        float part[kNormParts];
+#pragma unroll
+        for (int pp = 0; pp < kNormParts; ++pp) part[pp] = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < KH * 8; ++cc) {
+          const unsigned char* line = xbuf + (xb * KH + (cc >> 3)) * XBOX + row * 128;
+          const uint4 v = *reinterpret_cast<const uint4*>(line + (((cc & 7) ^ (row & 7)) << 4));
+          float f[8];
+          Vec16<__nv_bfloat16>::unpack(v, f);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) part[cc % kNormParts] = fmaf(f[k], f[k], part[cc % kNormParts]);
+        }
+#pragma unroll
+        for (int pp = 0; pp < kNormParts; ++pp) sst += part[pp];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(x_empty + xb);
+      for (int rl = first; rl < gr; rl += kHashEpiPerQuad) {
+        const int uu = u + rl;
+        const int ab = uu % S, uk = uu / S;
+        if (*abort_flag || !mbar_wait(acc_full + ab, uk & 1)) {
+          fail();
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tbase = tmem + tlane + ab * p.tmem_cols;
+        BatchLead st;
+        st.reset();
+        for (int b0 = 0; b0 < nbc; b0 += kHashMaxBatches) {
+          const int K = min(kHashMaxBatches, nbc - b0);
+          uint32_t V[kHashMaxBatches][16];
+#pragma unroll
+          for (int k = 0; k < kHashMaxBatches; ++k)
+            if (k < K) tmem_ld16(tbase + (b0 + k) * 16, V[k]);
+          tmem_wait_ld_regs(V);
+          if (b0 + kHashMaxBatches >= nbc) {  // the unit's last loads: release it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty + ab);
+          }
+#pragma unroll
+          for (int k = 0; k < kHashMaxBatches; ++k)
+            if (k < K) st.add(V[k], (float)((b0 + k) * 16));
+        }
+        float m1, m2, sv;
+        int idx;
+        st.finish(m1, m2, idx, sv);
+        if (t < a.n) hash_decide<D>(a, p, bh, t, r0 + rl, m1, m2, idx, sv, sst, rn_s[r0 + rl]);
+      }
+      u += gr;
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -542,7 +664,7 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
         BatchLead st;
         st.reset();
         for (int c = 0; ok && c < p.ch; ++c, ++u) {
-          const int ab = u & 1, uk = u >> 1;
+          const int ab = u % S, uk = u / S;
           if (!mbar_wait(acc_full + ab, uk & 1)) {
             fail();
             ok = false;
@@ -594,27 +716,10 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
             top2_merge(m1, m2, idx, sv, o.x, o.y, __float_as_int(o.z), o.w);
           }
           if (t < a.n) {
-            const int r = r0 + rl;
-            // ||x|| rounded up past the fp32 rounding of its square sum
             float sst = 0.f;
 #pragma unroll
             for (int o_ = 0; o_ < PO; ++o_) sst += sslot[o_ * 32];
-            if (a.pinv != nullptr && r == 0)  // once per token, from the first round
-              a.pinv[(int64_t)bh * a.n + t] = sst > 0.f ? 1.0f / sqrtf(sst) : 0.f;
-            const float xnorm = sqrtf(sst) * 1.0001f;
-            const float tau = kTieFactor * (float)D * 1.1920929e-7f * xnorm * rn_s[r];
-            const int bucket = idx + (sv < 0.f ? p.half : 0);
-            const int64_t at = ((int64_t)bh * a.rounds + r) * a.n + t;
-            a.buckets[at] = bucket;
-            if (a.hist != nullptr)  // the sort's tile histogram, counted here
-              atomicAdd(a.hist + ((int64_t)(bh * a.rounds + r) * a.nb + bucket) * a.sort_tiles +
-                            t / a.sort_tile,
-                        1);
-            if (!(m1 - m2 > tau)) {
-              atomicAdd(&a.hdr->hash_refined, 1u);
-              const uint32_t k = atomicAdd(&a.hdr->pad[16 + r], 1u);
-              a.refine[r * a.cap + k] = (uint64_t)((int64_t)bh * a.n + t);
-            }
+            hash_decide<D>(a, p, bh, t, r0 + rl, m1, m2, idx, sv, sst, rn_s[r0 + rl]);
           }
         }
       }
@@ -627,7 +732,7 @@ __global__ void __launch_bounds__(kHashWarps * 32, 1)
   // under a running MMA; the status word already records the timeout
   if (warp == 1 && !*drain_fail) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * p.tmem_cols);
+    tmem_dealloc(tmem, S * p.tmem_cols);
   }
 }
 

@@ -236,19 +236,12 @@ lsh_status launch_hash_tc(const Dims& D, const Layout& L, const void* x, const v
   if (per > a.tiles) per = a.tiles;
   a.ctas_per_group = per;
   const unsigned grid = (unsigned)(per * p.groups);
-  if (D.d == 64) {
-    auto kern = k_hash_tc<64>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) !=
-        cudaSuccess)
-      return LSH_ERR_CUDA;
-    kern<<<grid, kHashWarps * 32, p.smem, st>>>(tmx, tmr, a, p);
-  } else {
-    auto kern = k_hash_tc<128>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) !=
-        cudaSuccess)
-      return LSH_ERR_CUDA;
-    kern<<<grid, kHashWarps * 32, p.smem, st>>>(tmx, tmr, a, p);
-  }
+  auto kern = D.d == 64 ? (p.upw ? k_hash_tc<64, true> : k_hash_tc<64, false>)
+                        : (p.upw ? k_hash_tc<128, true> : k_hash_tc<128, false>);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) !=
+      cudaSuccess)
+    return LSH_ERR_CUDA;
+  kern<<<grid, kHashWarps * 32, p.smem, st>>>(tmx, tmr, a, p);
   if ((s = mark(ev, 2, st)) != LSH_OK) return s;
   // eight CTAs per SM over the rounds: a round's queue (a fraction of a percent
   // of its tokens) is one wave of 8-token batches; surplus CTAs exit at once
