@@ -76,6 +76,30 @@ def test_hash_full(w):
     check_buckets(got, ref, margin, w.name)
 
 
+# Epilogue forms of the tensor-core hash: a round of at most 128 projected
+# columns (b <= 256) is taken whole by one warp per quadrant, the warps taking
+# rounds in turn across tiles; wider rounds are split over the warps. These
+# cases cover one and two rounds per tile, rounds spread over several CTA
+# groups (16 rounds of resident R do not fit one CTA), and both head sizes.
+HASH_FORMS = [
+    I.LONG_64K.with_(name="h-d128-b256-R16", heads=2, n=16384, n_buckets=256, rounds=16),
+    I.LONG_64K.with_(name="h-d128-b256-R2", heads=2, n=16384, n_buckets=256, rounds=2),
+    I.LONG_64K.with_(name="h-d64-b32-R1", heads=3, n=16384, d=64, n_buckets=32, rounds=1),
+    I.LONG_64K.with_(name="h-d64-b128-R5", heads=2, n=8192 + 77, d=64, n_buckets=128, rounds=5),
+    I.LONG_64K.with_(name="h-d128-b512-R3", heads=2, n=16384, n_buckets=512, rounds=3),
+]
+
+
+@pytest.mark.parametrize("w", HASH_FORMS, ids=lambda w: w.name)
+def test_hash_epilogue_forms(w):
+    x, v = I.make_qkv(w)
+    R = I.make_rotations(w)
+    ref, margin = oracle.hash_all(x, R)
+    xg, Rg = to_gpu(x, R)
+    got = lb.lsh_attn_hash(xg, Rg, w.n_buckets).cpu().numpy()
+    check_buckets(got, ref, margin, w.name)
+
+
 @pytest.mark.parametrize("w", [I.LONG_64K, I.IMAGE_12K] + SWEEP_LARGE, ids=lambda w: w.name)
 def test_hash_sampled_tokens(w):
     """Full-size launch; the oracle re-derives a sample of (b, h, token) rows."""
