@@ -113,16 +113,19 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  unsigned char* xt = base;                                           // [2][KH][192][128 B]
-  unsigned char* vt = base + 2 * TILE;                                // [2][KH][192][128 B]
-  unsigned char* ostage = base + 4 * TILE;                            // [4 warps][32][128 B]
+  // tiles of x and of v in flight: three at d = 64 (small tiles), so a unit's
+  // rows can be gathered while the two before it are still in use
+  constexpr int NB = D == 64 ? 3 : 2;
+  unsigned char* xt = base;                                           // [NB][KH][192][128 B]
+  unsigned char* vt = base + NB * TILE;                               // [NB][KH][192][128 B]
+  unsigned char* ostage = base + 2 * NB * TILE;                       // [4 warps][32][128 B]
   float2* ktab = reinterpret_cast<float2*>(ostage + 4 * 32 * 128);    // [ring][192] (scale, pos)
   float* rstat = reinterpret_cast<float*>(ktab + kAttnRing * kAttnKeys);  // [4][128] 1/sum
   uint64_t* bars = reinterpret_cast<uint64_t*>(rstat + kAttnStats * 128);
-  uint64_t* xfull = bars + 0;    // [2] x rows landed (64 x-loader threads)
-  uint64_t* xfree = bars + 2;    // [2] S MMA done with the x tile
-  uint64_t* vfull = bars + 4;    // [2] v rows landed (64 v-loader threads)
-  uint64_t* vfree = bars + 6;    // [2] PV MMA done with the v tile
+  uint64_t* xfull = bars + 36;   // [NB] x rows landed (64 x-loader threads)
+  uint64_t* xfree = bars + 39;   // [NB] S MMA done with the x tile
+  uint64_t* vfull = bars + 42;   // [NB] v rows landed (64 v-loader threads)
+  uint64_t* vfree = bars + 45;   // [NB] PV MMA done with the v tile
   uint64_t* sfull = bars + 8;    // [2] S MMA done
   uint64_t* pready = bars + 10;  // [2] P written (4 softmax warps)
   uint64_t* sfree = bars + 12;   // [2] PV MMA done with P
@@ -149,11 +152,13 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
   if (nu == 0) return;  // uniform across the CTA
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NB; ++i) {
       mbar_init(xfull + i, 64);
       mbar_init(xfree + i, 1);
       mbar_init(vfull + i, 64);
       mbar_init(vfree + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(sfull + i, 1);
       mbar_init(pready + i, 4);
       mbar_init(sfree + i, 1);
@@ -280,12 +285,13 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     const int pair_bar = 2 + (xl ? 0 : 1);
     bool stopped = false;
     for (int i = 0; i < nu; ++i) {
-      const int s = i & 1, k = i >> 1, m = i & (kAttnRing - 1), km = i / kAttnRing;
+      const int s = i % NB, k = i / NB, m = i & (kAttnRing - 1), km = i / kAttnRing;
+      const int sp = (i + NB - 1) % NB;  // tile of unit i - 1
       bool got;
-      if (xl)  // ring slot m free (unit i - 4 done with it), x tile s free (S of unit i - 2)
+      if (xl)  // ring slot m free (unit i - 4 done with it), x tile s free (S of unit i - NB)
         got = (km == 0 || mbar_wait(mfree + m, (km - 1) & 1)) &&
               (k == 0 || mbar_wait(tfree + s, (k - 1) & 1));
-      else     // ring slot m written for unit i, v tile s free (PV of unit i - 2)
+      else     // ring slot m written for unit i, v tile s free (PV of unit i - NB)
         got = mbar_wait(mfull + m, km & 1) && (k == 0 || mbar_wait(tfree + s, (k - 1) & 1));
       if (!got) fail();
       // both warps of the pair stop together (a failure anywhere sets abort_flag)
@@ -328,7 +334,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
         cp_async_wait_prev();  // this thread's copies of unit i - 1 have landed
         if (carry) {
           bar_sync_any(pair_bar, 64, false);  // ... and the whole pair's
-          const unsigned char* prev = tiles + (s ^ 1) * TILE;
+          const unsigned char* prev = tiles + sp * TILE;
           // every piece is loaded before the first is stored (8 at a time)
           constexpr int NP = kAttnM * 8 * KH / 64;  // pieces per thread
 #pragma unroll
@@ -349,7 +355,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
           }
         }
         fence_proxy_async_smem();  // unit i - 1's rows (and unit i's carried ones) for the MMA
-        mbar_arrive(full + (s ^ 1));
+        mbar_arrive(full + sp);
       }
       u_prev = u_cur;
       u_cur = u_n1;
@@ -360,7 +366,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
     cp_async_wait_all();  // nothing of this thread's still writes shared memory at exit
     if (!stopped) {  // the last unit
       fence_proxy_async_smem();
-      mbar_arrive(full + ((nu - 1) & 1));
+      mbar_arrive(full + ((nu - 1) % NB));
     }
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
@@ -368,11 +374,12 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
       const uint32_t idesc_s = idesc_bf16_f32(128, kAttnKeys);
       const uint32_t idesc_o = idesc_bf16_f32(128, D) | (1u << 16);  // B = V, MN-major
       auto issue_s = [&](int i) {
-        const int s = i & 1, k = i >> 1;
-        if (!mbar_wait(xfull + s, k & 1)) return false;
+        const int s = i & 1, k = i >> 1;     // S in TMEM
+        const int tb = i % NB, tk = i / NB;  // x tile
+        if (!mbar_wait(xfull + tb, tk & 1)) return false;
         if (k > 0 && !mbar_wait(sfree + s, (k - 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t xa = smem_u32(xt + s * TILE);
+        const uint32_t xa = smem_u32(xt + tb * TILE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int kh = kk >> 2, ks = kk & 3;
@@ -381,23 +388,24 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
           mma_bf16_ss(tmem + s * 192, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(sfull + s);
-        mma_commit(xfree + s);
+        mma_commit(xfree + tb);
         return true;
       };
       auto issue_pv = [&](int i) {
-        const int s = i & 1, k = i >> 1;
+        const int s = i & 1, k = i >> 1;     // P in TMEM
+        const int tb = i % NB, tk = i / NB;  // v tile
         if (!mbar_wait(pready + s, k & 1)) return false;
-        if (!mbar_wait(vfull + s, k & 1)) return false;
+        if (!mbar_wait(vfull + tb, tk & 1)) return false;
         if (i > 0 && !mbar_wait(ofree, (i - 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t va = smem_u32(vt + s * TILE);
+        const uint32_t va = smem_u32(vt + tb * TILE);
 #pragma unroll
         for (int kk = 0; kk < kAttnKeys / 16; ++kk) {
           const uint64_t bd = desc_mnmajor_sw128(va + kk * 16 * 128, BOX);
           mma_bf16_ts(tm_o, tmem + s * 192 + kk * 8, bd, idesc_o, kk > 0 ? 1u : 0u);
         }
         mma_commit(ofull);
-        mma_commit(vfree + s);
+        mma_commit(vfree + tb);
         mma_commit(sfree + s);
         return true;
       };
@@ -585,8 +593,9 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 1)
 
 inline size_t attn_tc_smem(int D) {
   const size_t tile = (size_t)(D / 64) * kAttnKeys * 128;
-  return 1024 + 4 * tile + 4 * 32 * 128 + (size_t)kAttnRing * kAttnKeys * 8 +
-         kAttnStats * 128 * 4 + 256;
+  const int nb = D == 64 ? 3 : 2;  // NB of the kernel
+  return 1024 + 2 * nb * tile + 4 * 32 * 128 + (size_t)kAttnRing * kAttnKeys * 8 +
+         kAttnStats * 128 * 4 + 512;
 }
 
 // 1/||x|| of every row of x [rows][D] (bf16), for the attention's key scales
