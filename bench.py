@@ -56,8 +56,8 @@ NCU_WORKLOAD = I.LONG_64K.name
 NCU_TRAFFIC: dict = {
     "hash_mma": {"file": "hash_tc.cuh", "bytes": 150685952,
                  "sha256": "be5f804820c229310485427ca73d1d2fd51ddb948095ae8bbe20fc8be0cd7c14"},
-    "chunk_attention": {"file": "attn_tc.cuh", "bytes": 837818368,
-                 "sha256": "1e37f006eaa651e55be3ac720d1c9fc5d42506a6510905e847f7b9470872405a"},
+    "chunk_attention": {"file": "attn_tc.cuh", "bytes": 839529728,
+                 "sha256": "d9137349f2a4744965edacb7179a784ccd709fedbc7c1c0817532d3ace81986e"},
     "unsort_merge": {"file": "merge.cuh", "bytes": 673624320,
                  "sha256": "f313dd4622da3353060cb7b84324a099bfef2be35a4e693135b8674f34cd17db"},
     "hash_refine": {"file": "hash_tc.cuh", "bytes": 1660416,
