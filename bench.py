@@ -54,18 +54,18 @@ EXTRA_WORKLOADS = ("image-12k", "bf16-short", "sweep-n131072-r8-iso", "sweep-n20
 # of the file at capture time); see profiles/.
 NCU_WORKLOAD = I.LONG_64K.name
 NCU_TRAFFIC: dict = {
-    "hash_mma": {"file": "hash_tc.cuh", "bytes": 150685952,
-                 "sha256": "be5f804820c229310485427ca73d1d2fd51ddb948095ae8bbe20fc8be0cd7c14"},
+    "hash_mma": {"file": "hash_tc.cuh", "bytes": 150568448,
+                 "sha256": "12d5a1b8c7fa8d801e4068aa78d84d763a93a54e65660f0779ff448a785ab33d"},
     "chunk_attention": {"file": "attn_tc.cuh", "bytes": 839529728,
                  "sha256": "d9137349f2a4744965edacb7179a784ccd709fedbc7c1c0817532d3ace81986e"},
     "unsort_merge": {"file": "merge.cuh", "bytes": 673624320,
                  "sha256": "f313dd4622da3353060cb7b84324a099bfef2be35a4e693135b8674f34cd17db"},
-    "hash_refine": {"file": "hash_tc.cuh", "bytes": 1660416,
-                 "sha256": "be5f804820c229310485427ca73d1d2fd51ddb948095ae8bbe20fc8be0cd7c14"},
+    "hash_refine": {"file": "hash_tc.cuh", "bytes": 1661184,
+                 "sha256": "12d5a1b8c7fa8d801e4068aa78d84d763a93a54e65660f0779ff448a785ab33d"},
     "sort_rank": {"file": "sort.cuh", "bytes": 12597760,
                  "sha256": "e031792086f8fef697f441014adf16e9a9b36d922f1a623610bc2e5e46c4b5ab"},
     "hash_prep": {"file": "hash_tc.cuh", "bytes": 533760,
-                 "sha256": "be5f804820c229310485427ca73d1d2fd51ddb948095ae8bbe20fc8be0cd7c14"},
+                 "sha256": "12d5a1b8c7fa8d801e4068aa78d84d763a93a54e65660f0779ff448a785ab33d"},
     "sort_scan": {"file": "sort.cuh", "bytes": 4203776,
                  "sha256": "e031792086f8fef697f441014adf16e9a9b36d922f1a623610bc2e5e46c4b5ab"},
 }

@@ -280,47 +280,52 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 }
 
 // Top-two tracker of |p_j| over one token's columns, fed 16 columns at a
-// time. Per batch it takes the batch maximum (a tree of three-input max
-// operations) and keeps the whole batch only when that maximum leads; the
-// argmax, its sign and the largest value beside it are found once, in the
-// lead batch, when the round is done. The second largest |p| overall is the
-// larger of that in-batch value and the largest maximum of the other
-// batches, so the result equals a column-by-column top-two scan. Columns
+// time. Per batch it takes the maxima of the two 8-column halves (trees of
+// three-input max operations) and, only when the batch maximum leads, keeps
+// the leading half's signed values and the other half's maximum; the argmax,
+// its sign and the largest value beside it are found once, in the kept half,
+// when the round is done. The second largest |p| overall is the largest of
+// that in-half value, the other half's maximum and the largest maximum of the
+// other batches, so the result equals a column-by-column top-two scan. Ties
+// keep the lower columns (the earlier batch, then the lower half). Columns
 // past b/2 (zero rows of the padded rotation) give p = 0 exactly and never
 // lead: the first of equal maxima keeps the lead, and a zero maximum is a
 // tie that is re-decided.
 struct BatchLead {
-  float m1;     // largest |p| so far (-1 before the first batch)
-  float m2o;    // largest batch maximum outside the lead batch
-  float j0;     // first column of the lead batch (exact in fp32)
-  float s[16];  // the lead batch's signed values
+  float m1;    // largest |p| so far (-1 before the first batch)
+  float m2o;   // largest batch maximum outside the lead batch
+  float j0;    // first column of the kept half (exact in fp32)
+  float o;     // largest |p| of the lead batch's other half
+  float s[8];  // the kept half's signed values
   __device__ __forceinline__ void reset() {
     m1 = -1.f;
     m2o = 0.f;
     j0 = 0.f;
+    o = 0.f;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) s[k] = 0.f;
+    for (int k = 0; k < 8; ++k) s[k] = 0.f;
   }
   // Batch of 16 values starting at column jb.
   __device__ __forceinline__ void add(const uint32_t (&v)[16], float jb) {
     float w[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) w[k] = __uint_as_float(v[k]);
-    const float u0 = fmax3(fabsf(w[0]), fabsf(w[1]), fabsf(w[2]));
-    const float u1 = fmax3(fabsf(w[3]), fabsf(w[4]), fabsf(w[5]));
-    const float u2 = fmax3(fabsf(w[6]), fabsf(w[7]), fabsf(w[8]));
-    const float u3 = fmax3(fabsf(w[9]), fabsf(w[10]), fabsf(w[11]));
-    const float u4 = fmax3(fabsf(w[12]), fabsf(w[13]), fabsf(w[14]));
-    const float bm = fmaxf(fmax3(u0, u1, u2), fmax3(u3, u4, fabsf(w[15])));
+    const float lo = fmax3(fmax3(fabsf(w[0]), fabsf(w[1]), fabsf(w[2])),
+                           fmax3(fabsf(w[3]), fabsf(w[4]), fabsf(w[5])),
+                           fmaxf(fabsf(w[6]), fabsf(w[7])));
+    const float hi = fmax3(fmax3(fabsf(w[8]), fabsf(w[9]), fabsf(w[10])),
+                           fmax3(fabsf(w[11]), fabsf(w[12]), fabsf(w[13])),
+                           fmaxf(fabsf(w[14]), fabsf(w[15])));
+    const float bm = fmaxf(lo, hi);
     const bool lead = bm > m1;        // the earlier batch keeps the lead on a tie
     m2o = fmaxf(m2o, fminf(bm, m1));  // the batch that does not lead
     m1 = fmaxf(m1, bm);
-    // the copy is branched over rather than selected element by element:
-    // measured cheaper even when every lane leads
     if (lead) {
-      j0 = jb;
+      const bool up = hi > lo;  // the lower half keeps the lead on a tie
+      j0 = up ? jb + 8.f : jb;
+      o = fminf(lo, hi);
 #pragma unroll
-      for (int k = 0; k < 16; ++k) s[k] = w[k];
+      for (int k = 0; k < 8; ++k) s[k] = up ? w[8 + k] : w[k];
     }
   }
   // Largest |p|, second largest, argmax column and its signed value; all
@@ -329,7 +334,7 @@ struct BatchLead {
     float a1 = -1.f, a2 = 0.f, sv = 0.f;
     int k1 = 0;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
+    for (int k = 0; k < 8; ++k) {
       const float a = fabsf(s[k]);
       const bool gt = a > a1;  // lowest column on a tie
       a2 = gt ? fmaxf(a2, a1) : fmaxf(a2, a);
@@ -344,7 +349,7 @@ struct BatchLead {
       osv = 0.f;
     } else {
       om1 = a1;
-      om2 = fmaxf(a2, m2o);
+      om2 = fmaxf(fmaxf(a2, o), m2o);
       oidx = (int)j0 + k1;
       osv = sv;
     }
